@@ -1,0 +1,213 @@
+"""CPU oracle for group-wise INT4 quantization and the W4A16 decode product.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  The product library never loads it and shares no code with it.
+
+The arithmetic lives in ``q4_oracle.c`` (plain single-threaded C11, IEEE fp32
+for the quantizer as the pages state it, fp64 for the products); this module
+only compiles it with gcc on first use and marshals numpy arrays.
+
+Functions with no independent pin beyond their definition are listed in the
+header of ``q4_oracle.c``; every function here is pinned by
+``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import tempfile
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "q4_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "libq4oracle.so")
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+          "-fvisibility=hidden", "-Wall", "-Wextra"]
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library (idempotent); returns its path."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    os.makedirs(_BUILD, exist_ok=True)
+    fd, tmp = tempfile.mkstemp(suffix=".so", dir=_BUILD)
+    os.close(fd)
+    subprocess.run(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"], check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    P = ctypes.c_void_p
+    I64 = ctypes.c_int64
+    I32 = ctypes.c_int32
+    lib.oracle_f16_to_f32.argtypes = [ctypes.c_uint16]
+    lib.oracle_f16_to_f32.restype = ctypes.c_float
+    lib.oracle_f32_to_f16.argtypes = [ctypes.c_float]
+    lib.oracle_f32_to_f16.restype = ctypes.c_uint16
+    lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+    lib.oracle_bf16_to_f32.restype = ctypes.c_float
+    lib.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
+    lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
+    for name in ("oracle_f16_to_f32_n", "oracle_f32_to_f16_n", "oracle_bf16_to_f32_n",
+                 "oracle_f32_to_bf16_n"):
+        getattr(lib, name).argtypes = [P, P, I64]
+        getattr(lib, name).restype = None
+    lib.oracle_quantize_value.argtypes = [ctypes.c_float, ctypes.c_float, I32, I32, I32]
+    lib.oracle_quantize_value.restype = I32
+    lib.oracle_quantize_pack.argtypes = [P, I64, I64, I32, I32, P, P, P]
+    lib.oracle_quantize_pack.restype = ctypes.c_int
+    lib.oracle_code_at.argtypes = [P, I64, I64, I64, I32]
+    lib.oracle_code_at.restype = I32
+    lib.oracle_dequant_f32.argtypes = [P, P, P, I64, I64, I32, I32, P]
+    lib.oracle_dequant_f32.restype = ctypes.c_int
+    lib.oracle_gemv_rows_f64.argtypes = [P, P, P, I64, I64, I32, I32, P, I64, P, I64, P]
+    lib.oracle_gemv_rows_f64.restype = ctypes.c_int
+    lib.oracle_gemv_f64.argtypes = [P, P, P, I64, I64, I32, I32, P, I64, P]
+    lib.oracle_gemv_f64.restype = ctypes.c_int
+    lib.oracle_dense_rows_f64.argtypes = [P, I64, I64, P, I64, P, I64, P]
+    lib.oracle_dense_rows_f64.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# ----------------------------------------------------------------- codecs
+
+def f16_to_f32(h: int) -> float:
+    return _load().oracle_f16_to_f32(int(h))
+
+
+def f32_to_f16(f: float) -> int:
+    return _load().oracle_f32_to_f16(float(f))
+
+
+def bf16_to_f32(b: int) -> float:
+    return _load().oracle_bf16_to_f32(int(b))
+
+
+def f32_to_bf16(f: float) -> int:
+    return _load().oracle_f32_to_bf16(float(f))
+
+
+def _codec_n(fn: str, a: np.ndarray, in_dtype, out_dtype) -> np.ndarray:
+    src = np.ascontiguousarray(a, dtype=in_dtype)
+    dst = np.empty(src.shape, dtype=out_dtype)
+    getattr(_load(), fn)(_ptr(src), _ptr(dst), src.size)
+    return dst
+
+
+def f16_bits_to_f32_array(h: np.ndarray) -> np.ndarray:
+    """Element-wise oracle fp16 decode of a uint16 array."""
+    return _codec_n("oracle_f16_to_f32_n", h, np.uint16, np.float32)
+
+
+def f32_to_f16_bits_array(f: np.ndarray) -> np.ndarray:
+    """Element-wise oracle fp32 -> fp16 (round to nearest even) encode."""
+    return _codec_n("oracle_f32_to_f16_n", f, np.float32, np.uint16)
+
+
+def bf16_bits_to_f32_array(b: np.ndarray) -> np.ndarray:
+    return _codec_n("oracle_bf16_to_f32_n", b, np.uint16, np.float32)
+
+
+def f32_to_bf16_bits_array(f: np.ndarray) -> np.ndarray:
+    return _codec_n("oracle_f32_to_bf16_n", f, np.float32, np.uint16)
+
+
+def quantize_value(w: float, s: float, z: int, qmin: int, qmax: int) -> int:
+    """clamp(rne(w / s) + z, qmin, qmax) with an fp32 scale s."""
+    return _load().oracle_quantize_value(float(w), float(s), int(z), int(qmin), int(qmax))
+
+
+# -------------------------------------------------------------- quantizer
+
+def quantize_pack(W: np.ndarray, group_size: int, symmetric: bool):
+    """W: [out, in] float32 (exact values of fp16/bf16 weights).
+
+    Returns (qweight uint8 [out, in/2], scales uint16 fp16-bits [out, in/g],
+    zeros uint16 fp16-bits [out, in/g] or None)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    out, inn = W.shape
+    G = inn // group_size
+    q = np.zeros((out, inn // 2), dtype=np.uint8)
+    s = np.zeros((out, G), dtype=np.uint16)
+    z = None if symmetric else np.zeros((out, G), dtype=np.uint16)
+    rc = _load().oracle_quantize_pack(_ptr(W), out, inn, int(group_size), int(bool(symmetric)),
+                                      _ptr(q), _ptr(s), _ptr(z))
+    if rc != 0:
+        raise ValueError("oracle_quantize_pack rejected its arguments")
+    return q, s, z
+
+
+def code_at(qweight: np.ndarray, inn: int, r: int, k: int, symmetric: bool) -> int:
+    return _load().oracle_code_at(_ptr(np.ascontiguousarray(qweight)), inn, r, k, int(symmetric))
+
+
+def dequant(qweight, scales, zeros, out: int, inn: int, group_size: int, symmetric: bool):
+    """Returns W_hat [out, in] float32 = s * (q - z) (exact in fp32)."""
+    qweight = np.ascontiguousarray(qweight, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    zeros = None if zeros is None else np.ascontiguousarray(zeros, dtype=np.uint16)
+    W_hat = np.empty((out, inn), dtype=np.float32)
+    rc = _load().oracle_dequant_f32(_ptr(qweight), _ptr(scales), _ptr(zeros), out, inn,
+                                    int(group_size), int(bool(symmetric)), _ptr(W_hat))
+    if rc != 0:
+        raise ValueError("oracle_dequant_f32 rejected its arguments")
+    return W_hat
+
+
+def gemv(qweight, scales, zeros, out: int, inn: int, group_size: int, symmetric: bool,
+         x: np.ndarray, rows=None) -> np.ndarray:
+    """y [B, len(rows)] fp64 = x . W_hat^T over the given rows (all if None).
+
+    x: [B, in] float (exact values of the bf16/fp16 activations)."""
+    qweight = np.ascontiguousarray(qweight, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    zeros = None if zeros is None else np.ascontiguousarray(zeros, dtype=np.uint16)
+    x = np.ascontiguousarray(np.atleast_2d(x), dtype=np.float64)
+    B = x.shape[0]
+    if rows is None:
+        rows = np.arange(out, dtype=np.int64)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    y = np.empty((B, rows.shape[0]), dtype=np.float64)
+    rc = _load().oracle_gemv_rows_f64(_ptr(qweight), _ptr(scales), _ptr(zeros), out, inn,
+                                      int(group_size), int(bool(symmetric)), _ptr(x), B,
+                                      _ptr(rows), rows.shape[0], _ptr(y))
+    if rc != 0:
+        raise ValueError("oracle_gemv_rows_f64 rejected its arguments")
+    return y
+
+
+def dense(W: np.ndarray, x: np.ndarray, rows=None) -> np.ndarray:
+    """y [B, len(rows)] fp64 = x . W^T for float32 W (exact bf16 values)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    out, inn = W.shape
+    x = np.ascontiguousarray(np.atleast_2d(x), dtype=np.float64)
+    B = x.shape[0]
+    if rows is None:
+        rows = np.arange(out, dtype=np.int64)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    y = np.empty((B, rows.shape[0]), dtype=np.float64)
+    rc = _load().oracle_dense_rows_f64(_ptr(W), out, inn, _ptr(x), B, _ptr(rows),
+                                       rows.shape[0], _ptr(y))
+    if rc != 0:
+        raise ValueError("oracle_dense_rows_f64 rejected its arguments")
+    return y

@@ -1,0 +1,326 @@
+/*
+ * q4_oracle.c -- CPU oracle for group-wise INT4 weight quantization and the
+ * W4A16 matrix-vector product.  TEST INFRASTRUCTURE ONLY: nothing on the
+ * product path may link, load or call this file.  Only tests/, the smoke
+ * check in __graft_entry__.py and the cpu_baseline / reference legs of
+ * bench.py use it.
+ *
+ * Plain, single-threaded C11.  No CUDA headers, no code shared with the GPU
+ * library.  Compiled without -ffast-math and with -ffp-contract=off so that
+ * every fp32 operation below is one IEEE-754 binary32 operation rounded to
+ * nearest-even, exactly as written.
+ *
+ * What it computes, and where the pages define it:
+ *
+ *  - the affine quantizer  q = clamp(round(w/s) + z, qmin, qmax),
+ *    dequant  w_hat = s * (q - z)
+ *      "LLM 后训练量化深度实战" (ybb.press), section 二, first equation;
+ *      arganzheng.life post-training-quantization-gptq-awq-and-rotation,
+ *      section 二.2 (基本形式与粒度), first equation;
+ *      "量化：PTQ、GPTQ、AWQ 与 SmoothQuant" (charles2530.github.io),
+ *      section 1 (量化的统一形式).
+ *  - symmetric scale s = max|w| / (2^(b-1) - 1) = amax / 7 with z = 0, and
+ *    asymmetric scale s = (max - min) / (2^b - 1) = (max - min) / 15 with an
+ *    integer zero-point z: arganzheng.life, section 二.2.
+ *  - group-wise granularity along in_features, symmetric INT4 range [-8, 7]:
+ *    ybb.press, section 二, function quantize_per_group;
+ *    charles2530.github.io, section 1 (q in {-8..7}).
+ *  - zero-point as the integer code of real 0, z = round(-min / s):
+ *    arganzheng.life section 二.2 (z is added on the integer side);
+ *    "压缩算法" (cs-knowledge-wiki), section 7.4.1.1 (INT8 asymmetric form).
+ *  - two 4-bit codes per byte: "压缩算法" section 7.4.1.2 (pack_int4).
+ *  - the decode product y = x W^T of the dequantised weights:
+ *    arganzheng.life section 二.1 ([B,k] x [k,n] decode GEMM) and 二.3.
+ *
+ * Readings taken where the pages leave a step open (all listed in the design doc):
+ *  - the scale is computed in fp32 (IEEE division), stored as fp16, and the
+ *    STORED fp16 scale is the one that quantizes and dequantizes;
+ *  - round() is round-half-to-even (torch.round in the ybb.press code);
+ *  - a group whose stored scale is 0 gets all codes 0 (sym) / z = 0 (asym);
+ *  - asymmetric: z = clamp(rne(-min / s), 0, 15), stored as an fp16 integer;
+ *    codes are clamp(rne(w / s) + z, 0, 15);
+ *  - packing: element 2j in the low nibble of byte j, element 2j+1 in the
+ *    high nibble; symmetric codes stored as two's complement (q & 0xF).
+ *
+ * fp16 and bf16 codecs are written from the IEEE-754 binary16 definition and
+ * from bfloat16 = the upper 16 bits of binary32 (round to nearest even).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_API __attribute__((visibility("default")))
+
+/* ------------------------------------------------------------------ codecs */
+
+static uint32_t f32_bits(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+static float bits_f32(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+
+/* binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+ORACLE_API float oracle_f16_to_f32(uint16_t h) {
+    uint32_t sign = (uint32_t)(h >> 15) & 1u;
+    uint32_t exp = (uint32_t)(h >> 10) & 0x1Fu;
+    uint32_t frac = (uint32_t)h & 0x3FFu;
+    float mag;
+    if (exp == 0x1F) {
+        mag = frac ? NAN : INFINITY;
+    } else if (exp == 0) {
+        mag = ldexpf((float)frac, -24);            /* subnormal: frac * 2^-24 */
+    } else {
+        mag = ldexpf((float)(frac | 0x400u), (int)exp - 25); /* 1.f * 2^(e-15) */
+    }
+    return sign ? -mag : mag;
+}
+
+/* Round a binary32 value to the nearest binary16 value, ties to even.
+ * Works on the exact value: v = m * 2^e with a 24-bit integer m. */
+ORACLE_API uint16_t oracle_f32_to_f16(float f) {
+    uint32_t u = f32_bits(f);
+    uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+    uint32_t exp = (u >> 23) & 0xFFu;
+    uint32_t frac = u & 0x7FFFFFu;
+    if (exp == 0xFF) return (uint16_t)(sign | 0x7C00u | (frac ? 0x200u : 0u));
+    if (exp == 0 && frac == 0) return sign;
+    /* exact value = mant * 2^(e2) with mant < 2^24 */
+    uint32_t mant = exp ? (frac | 0x800000u) : frac;
+    int e2 = exp ? (int)exp - 150 : -149;
+    /* binary16 quantum for this magnitude: representable values are
+     * k * 2^q with q = max(unbiased_exp - 10, -24), unbiased exponent of the
+     * result computed from the leading bit of mant. */
+    int lead = 31 - __builtin_clz(mant);          /* position of leading 1 */
+    int unb = lead + e2;                          /* floor(log2 |v|) */
+    int q = unb - 10;
+    if (q < -24) q = -24;
+    int shift = q - e2;                           /* bits to drop from mant */
+    uint64_t k;
+    if (shift <= 0) {
+        k = (uint64_t)mant << (-shift);
+    } else if (shift > 40) {
+        k = 0;
+    } else {
+        uint64_t m = mant;
+        uint64_t kq = m >> shift;
+        uint64_t rem = m - (kq << shift);
+        uint64_t half = 1ull << (shift - 1);
+        if (rem > half || (rem == half && (kq & 1ull))) kq += 1;
+        k = kq;
+    }
+    /* value = k * 2^q; encode */
+    if (k == 0) return sign;
+    /* k may have overflowed into 2^11 after rounding: renormalise */
+    while (k >= 2048) { k >>= 1; q += 1; }    /* k even here, exact */
+    if (q == -24 && k < 1024) return (uint16_t)(sign | (uint16_t)k); /* subnormal */
+    /* normal: k in [1024, 2047], value = k * 2^q = 1.f * 2^(q+10) */
+    int be = q + 10 + 15;
+    if (be >= 31) return (uint16_t)(sign | 0x7C00u);  /* overflow -> inf */
+    return (uint16_t)(sign | (uint16_t)(be << 10) | (uint16_t)(k - 1024));
+}
+
+ORACLE_API float oracle_bf16_to_f32(uint16_t b) { return bits_f32((uint32_t)b << 16); }
+
+ORACLE_API uint16_t oracle_f32_to_bf16(float f) {
+    uint32_t u = f32_bits(f);
+    if (((u >> 23) & 0xFFu) == 0xFFu && (u & 0x7FFFFFu)) return (uint16_t)((u >> 16) | 0x40u);
+    uint32_t lower = u & 0xFFFFu;
+    uint32_t upper = u >> 16;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1; /* may carry into inf: correct */
+    return (uint16_t)upper;
+}
+
+/* array forms of the codecs (n elements) */
+ORACLE_API void oracle_f16_to_f32_n(const uint16_t* h, float* f, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) f[i] = oracle_f16_to_f32(h[i]);
+}
+ORACLE_API void oracle_f32_to_f16_n(const float* f, uint16_t* h, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) h[i] = oracle_f32_to_f16(f[i]);
+}
+ORACLE_API void oracle_bf16_to_f32_n(const uint16_t* b, float* f, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) f[i] = oracle_bf16_to_f32(b[i]);
+}
+ORACLE_API void oracle_f32_to_bf16_n(const float* f, uint16_t* b, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) b[i] = oracle_f32_to_bf16(f[i]);
+}
+
+/* ---------------------------------------------------------------- rounding */
+
+/* round half to even of a binary32 value (default IEEE rounding mode). */
+static float rne(float v) { return nearbyintf(v); }
+
+/* q = clamp(rne(w / s) + z, qmin, qmax): the affine quantizer of one value
+ * with an externally supplied fp32 scale (the worked rounding and clipping
+ * examples of "模型量化技术工程实践" (iopencloud.com), section 1.2, use it). */
+ORACLE_API int32_t oracle_quantize_value(float w, float s, int32_t z, int32_t qmin, int32_t qmax) {
+    float t = rne(w / s);                       /* IEEE fp32 division, RN */
+    /* add z and clamp in float, where t is an exact integer-valued float */
+    float v = t + (float)z;
+    if (!(v >= (float)qmin)) v = (float)qmin;   /* also maps NaN to qmin */
+    if (v > (float)qmax) v = (float)qmax;
+    return (int32_t)v;
+}
+
+/* -------------------------------------------------------------- quantizer */
+
+/*
+ * Group-wise INT4 round-to-nearest quantization and packing.
+ *   W        [out, in] fp32 values (the exact values of the fp16/bf16 input)
+ *   qweight  [out, in/2] bytes, element 2j low nibble, 2j+1 high nibble
+ *   scales   [out, in/g] fp16 bit patterns
+ *   zeros    [out, in/g] fp16 bit patterns (integer-valued), NULL iff symmetric
+ * Returns 0, or -1 on bad arguments (g not dividing in, g or in odd).
+ */
+ORACLE_API int oracle_quantize_pack(const float* W, int64_t out, int64_t in, int32_t g,
+                                    int32_t symmetric, uint8_t* qweight, uint16_t* scales,
+                                    uint16_t* zeros) {
+    if (g <= 0 || in <= 0 || out < 0 || (in % g) != 0 || (g % 2) != 0) return -1;
+    if (!symmetric && zeros == NULL) return -1;
+    const int64_t G = in / g;
+    int32_t* codes = (int32_t*)malloc(sizeof(int32_t) * (size_t)g);
+    if (!codes) return -1;
+    for (int64_t r = 0; r < out; ++r) {
+        for (int64_t j = 0; j < G; ++j) {
+            const float* w = W + r * in + j * g;
+            uint16_t s16;
+            float sf;
+            int32_t z = 0;
+            if (symmetric) {
+                /* a = max |w| over the group; s = a / 7 (2^(b-1) - 1 = 7) */
+                float a = 0.0f;
+                for (int32_t k = 0; k < g; ++k) {
+                    float m = fabsf(w[k]);
+                    if (m > a) a = m;
+                }
+                float s32 = a / 7.0f;
+                s16 = oracle_f32_to_f16(s32);
+                sf = oracle_f16_to_f32(s16);
+                for (int32_t k = 0; k < g; ++k)
+                    codes[k] = (sf == 0.0f) ? 0 : oracle_quantize_value(w[k], sf, 0, -8, 7);
+            } else {
+                /* s = (max - min) / 15, z = clamp(rne(-min / s), 0, 15) */
+                float mn = w[0], mx = w[0];
+                for (int32_t k = 1; k < g; ++k) {
+                    if (w[k] < mn) mn = w[k];
+                    if (w[k] > mx) mx = w[k];
+                }
+                float s32 = (mx - mn) / 15.0f;
+                s16 = oracle_f32_to_f16(s32);
+                sf = oracle_f16_to_f32(s16);
+                if (sf == 0.0f) {
+                    z = 0;
+                    for (int32_t k = 0; k < g; ++k) codes[k] = 0;
+                } else {
+                    z = oracle_quantize_value(-mn, sf, 0, 0, 15);
+                    for (int32_t k = 0; k < g; ++k)
+                        codes[k] = oracle_quantize_value(w[k], sf, z, 0, 15);
+                }
+                zeros[r * G + j] = oracle_f32_to_f16((float)z);
+            }
+            scales[r * G + j] = s16;
+            /* pack: two codes per byte, even element in the low nibble */
+            uint8_t* dst = qweight + r * (in / 2) + j * (g / 2);
+            for (int32_t k = 0; k < g; k += 2) {
+                uint8_t lo = (uint8_t)(codes[k] & 0xF);
+                uint8_t hi = (uint8_t)(codes[k + 1] & 0xF);
+                dst[k / 2] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+    }
+    free(codes);
+    return 0;
+}
+
+/* Unpack one code: low nibble for even k, high for odd k; symmetric codes are
+ * two's complement 4-bit integers, asymmetric codes are unsigned. */
+ORACLE_API int32_t oracle_code_at(const uint8_t* qweight, int64_t in, int64_t r, int64_t k,
+                                  int32_t symmetric) {
+    uint8_t b = qweight[r * (in / 2) + k / 2];
+    int32_t n = (k & 1) ? (b >> 4) : (b & 0xF);
+    if (symmetric && n >= 8) n -= 16;
+    return n;
+}
+
+/*
+ * Dequantisation w_hat = s * (q - z), in fp32.  The product of an fp16 scale
+ * (11 significant bits) and an integer of magnitude <= 15 is exact in fp32.
+ * W_hat [out, in] fp32.
+ */
+ORACLE_API int oracle_dequant_f32(const uint8_t* qweight, const uint16_t* scales,
+                                  const uint16_t* zeros, int64_t out, int64_t in, int32_t g,
+                                  int32_t symmetric, float* W_hat) {
+    if (g <= 0 || (in % g) != 0 || (g % 2) != 0) return -1;
+    if (!symmetric && zeros == NULL) return -1;
+    const int64_t G = in / g;
+    for (int64_t r = 0; r < out; ++r) {
+        for (int64_t k = 0; k < in; ++k) {
+            int64_t j = k / g;
+            float sf = oracle_f16_to_f32(scales[r * G + j]);
+            int32_t z = symmetric ? 0 : (int32_t)oracle_f16_to_f32(zeros[r * G + j]);
+            int32_t q = oracle_code_at(qweight, in, r, k, symmetric);
+            W_hat[r * in + k] = sf * (float)(q - z);
+        }
+    }
+    return 0;
+}
+
+/*
+ * y[b, i] = sum_k w_hat[rows[i], k] * x[b, k] in fp64, for a list of rows.
+ *   x [B, in] fp64 (exact values of the bf16/fp16 activations)
+ *   y [B, nrows] fp64
+ * The dequantised weights are exact in fp64; only the summation rounds.
+ */
+ORACLE_API int oracle_gemv_rows_f64(const uint8_t* qweight, const uint16_t* scales,
+                                    const uint16_t* zeros, int64_t out, int64_t in, int32_t g,
+                                    int32_t symmetric, const double* x, int64_t B,
+                                    const int64_t* rows, int64_t nrows, double* y) {
+    if (g <= 0 || (in % g) != 0 || (g % 2) != 0) return -1;
+    if (!symmetric && zeros == NULL) return -1;
+    const int64_t G = in / g;
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t r = rows[i];
+        if (r < 0 || r >= out) return -1;
+        for (int64_t b = 0; b < B; ++b) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < in; ++k) {
+                int64_t j = k / g;
+                double sf = (double)oracle_f16_to_f32(scales[r * G + j]);
+                double z = symmetric ? 0.0 : (double)oracle_f16_to_f32(zeros[r * G + j]);
+                double q = (double)oracle_code_at(qweight, in, r, k, symmetric);
+                acc += sf * (q - z) * x[b * in + k];
+            }
+            y[b * nrows + i] = acc;
+        }
+    }
+    return 0;
+}
+
+/* All rows: y [B, out]. */
+ORACLE_API int oracle_gemv_f64(const uint8_t* qweight, const uint16_t* scales,
+                               const uint16_t* zeros, int64_t out, int64_t in, int32_t g,
+                               int32_t symmetric, const double* x, int64_t B, double* y) {
+    int64_t* rows = (int64_t*)malloc(sizeof(int64_t) * (size_t)(out > 0 ? out : 1));
+    if (!rows) return -1;
+    for (int64_t r = 0; r < out; ++r) rows[r] = r;
+    int rc = oracle_gemv_rows_f64(qweight, scales, zeros, out, in, g, symmetric, x, B, rows, out, y);
+    free(rows);
+    return rc;
+}
+
+/*
+ * The unquantised reference product y[b, i] = sum_k W[rows[i], k] * x[b, k]
+ * in fp64, for W given as exact fp32 values (of bf16 weights).  This is the
+ * bf16 decode matmul the INT4 path is compared with (ybb.press section 一,
+ * roofline_bound example; arganzheng.life section 二.4 batch table).
+ */
+ORACLE_API int oracle_dense_rows_f64(const float* W, int64_t out, int64_t in, const double* x,
+                                     int64_t B, const int64_t* rows, int64_t nrows, double* y) {
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t r = rows[i];
+        if (r < 0 || r >= out) return -1;
+        for (int64_t b = 0; b < B; ++b) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < in; ++k) acc += (double)W[r * in + k] * x[b * in + k];
+            y[b * nrows + i] = acc;
+        }
+    }
+    return 0;
+}

@@ -1,0 +1,107 @@
+"""Seeded synthetic inputs: weight matrices, activation batches and the layer
+shapes of the benchmarked decode linears.
+
+This module holds only random-number recipes and shapes -- none of the
+quantization arithmetic -- so that the CUDA path and the CPU oracle can be fed
+identical inputs without sharing any method code.
+
+Shapes are those of Llama-3-8B and Llama-3-70B decoder linears ([out, in],
+W row-major, y = x W^T); weight statistics follow the pages' examples
+(N(0, 0.02^2) fp16 weights in the quantize_per_group example of "LLM 后训练量化
+深度实战", section 二) and a heavy-tailed variant (0.02 * Student-t with 3
+degrees of freedom, clipped at +-1) for the heavy-tail discussion of
+arganzheng.life post-training-quantization-gptq-awq-and-rotation, section 四.1.
+"""
+from __future__ import annotations
+
+import torch
+
+# Llama-3-8B decoder linears: name -> (out, in)
+LLAMA3_8B = {
+    "q_proj": (4096, 4096),
+    "k_proj": (1024, 4096),
+    "v_proj": (1024, 4096),
+    "o_proj": (4096, 4096),
+    "gate_proj": (14336, 4096),
+    "up_proj": (14336, 4096),
+    "down_proj": (4096, 14336),
+}
+LLAMA3_8B_LAYERS = 32
+
+# Llama-3-70B decoder linears: name -> (out, in)
+LLAMA3_70B = {
+    "q_proj": (8192, 8192),
+    "k_proj": (1024, 8192),
+    "v_proj": (1024, 8192),
+    "o_proj": (8192, 8192),
+    "gate_proj": (28672, 8192),
+    "up_proj": (28672, 8192),
+    "down_proj": (8192, 28672),
+}
+LLAMA3_70B_LAYERS = 80
+LLAMA3_70B_MLP = ("gate_proj", "up_proj", "down_proj")
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def normal_weight(out: int, inn: int, seed: int, std: float = 0.02,
+                  device="cpu") -> torch.Tensor:
+    """W = (N(0,1) * std).half(), [out, in]."""
+    g = _gen(seed, device)
+    w = torch.randn(out, inn, generator=g, device=device, dtype=torch.float32)
+    return (w * std).to(torch.float16)
+
+
+def student_t_weight(out: int, inn: int, seed: int, std: float = 0.02, df: int = 3,
+                     clip: float = 1.0, device="cpu") -> torch.Tensor:
+    """W = clamp(std * t_df, -clip, clip).half() with t_df = z / sqrt(chi2_df / df),
+    chi2_df the sum of df squared standard normals."""
+    g = _gen(seed, device)
+    z = torch.randn(out, inn, generator=g, device=device, dtype=torch.float32)
+    chi2 = torch.zeros(out, inn, device=device, dtype=torch.float32)
+    for _ in range(df):
+        u = torch.randn(out, inn, generator=g, device=device, dtype=torch.float32)
+        chi2.add_(u * u)
+    t = z / torch.sqrt(chi2 / df)
+    return torch.clamp(t * std, -clip, clip).to(torch.float16)
+
+
+def uniform_weight(out: int, inn: int, seed: int, amp: float = 0.05,
+                   device="cpu") -> torch.Tensor:
+    """W ~ U(-amp, amp) fp16."""
+    g = _gen(seed, device)
+    w = torch.rand(out, inn, generator=g, device=device, dtype=torch.float32)
+    return ((w * 2 - 1) * amp).to(torch.float16)
+
+
+def activations(B: int, inn: int, seed: int, dtype=torch.bfloat16, n_outliers: int = 0,
+                outlier_seed: int | None = None, outlier_scale: float = 20.0,
+                device="cpu") -> torch.Tensor:
+    """x = N(0,1) [B, in] in ``dtype``; optionally ``n_outliers`` fixed input
+    channels (the first of a seeded permutation) scaled by ``outlier_scale``."""
+    g = _gen(seed, device)
+    x = torch.randn(B, inn, generator=g, device=device, dtype=torch.float32)
+    if n_outliers:
+        gp = _gen(outlier_seed if outlier_seed is not None else seed + 1, "cpu")
+        ch = torch.randperm(inn, generator=gp)[:n_outliers].to(device)
+        x[:, ch] *= outlier_scale
+    return x.to(dtype)
+
+
+def outlier_channels(inn: int, n_outliers: int, outlier_seed: int) -> torch.Tensor:
+    gp = _gen(outlier_seed, "cpu")
+    return torch.randperm(inn, generator=gp)[:n_outliers]
+
+
+def llama3_8b_layer_seeds(layer: int) -> dict:
+    """Distinct seeds for the seven linears of one layer (10..16 for layer 0)."""
+    return {name: 10 + 7 * layer + i for i, name in enumerate(LLAMA3_8B)}
+
+
+def llama3_70b_stack_seed(layer: int, idx: int) -> int:
+    """Seed of linear ``idx`` (0..6 in LLAMA3_70B order) of layer ``layer``."""
+    return 1000 * layer + idx
