@@ -1,0 +1,420 @@
+"""Benchmark of the W4A16 decode path on B200.
+
+Default workload (one "step"): the W4A16 products of a Llama-3-8B decode
+step at batch 1 -- q, k, v, o, gate, up, down of 32 distinct decoder layers
+(224 packed INT4 matrices, symmetric, group 128, 3.6 GB of codes + scales, so
+no step finds its weights in the 126 MB L2).  Weights are random N(0, 0.02^2)
+fp16 generated on the device from seeds, quantized with q4_quantize_pack and
+the fp16 copies freed; activations are bf16 N(0, 1).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload llama3-8b | llama3-70b-stack | sweep]
+
+Prints one JSON line (rank 0).  ``value`` is the aggregate HBM throughput of
+the INT4 products (algorithmic bytes / device time, CUDA events, max over
+ranks); ``us_per_layer`` the time of one decoder layer's seven products.
+With --gpus N > 1 (launched by torchrun) every rank runs its own independent
+replica of the workload (weak scaling, no collective in the timed region).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A16 GEMV µs/layer + HBM GB/s (% of B200 peak) at B=1; INT4/bf16 speedup vs B"
+UNIT = "GB/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algo_bytes(out, inn, g, B, sym=True):
+    """Bytes a W4A16 product must move: codes + scales (+ zeros) + x + y."""
+    meta = out * (inn // g) * 2 * (1 if sym else 2)
+    return out * inn // 2 + meta + B * inn * 2 + B * out * 2
+
+
+def dense_bytes(out, inn, B):
+    return out * inn * 2 + B * inn * 2 + B * out * 2
+
+
+def quant_bytes(out, inn, g, sym=True):
+    return out * inn * 2 + out * inn // 2 + out * (inn // g) * 2 * (1 if sym else 2)
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- workload
+def build_llama3_8b(q4, wl, torch, layers, rank, B, device):
+    """Quantized weights of `layers` distinct Llama-3-8B layers (sym g128)."""
+    mats = []
+    for layer in range(layers):
+        seeds = wl.llama3_8b_layer_seeds(layer + 1000 * rank)
+        for name, (out, inn) in wl.LLAMA3_8B.items():
+            W = wl.normal_weight(out, inn, seeds[name], device=device)
+            mats.append((name, q4.q4_quantize_pack(W, 128, True)))
+            del W
+    xs = {inn: wl.activations(B, inn, 17 + inn, device=device)
+          for inn in sorted({i for _, i in wl.LLAMA3_8B.values()})}
+    ys = {name: torch.empty(B, out, dtype=torch.bfloat16, device=device)
+          for name, (out, _) in wl.LLAMA3_8B.items()}
+    torch.cuda.synchronize()
+    return mats, xs, ys
+
+
+def time_region(torch, fn, steps, warmup, stream):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)  # ms
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import post_weight_quantization_group_b200 as q4
+    from post_weight_quantization_group_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    q4.load_library()
+    peaks, peak_kind = load_peaks()
+    stream = torch.cuda.current_stream()
+    B = 1
+    layers = args.layers
+    mats, xs, ys = build_llama3_8b(q4, wl, torch, layers, rank, B, device)
+    shapes = wl.LLAMA3_8B
+    step_bytes = sum(algo_bytes(*shapes[n], 128, B) for n, _ in mats)
+    launches_per_step = len(mats)
+
+    def step():
+        for name, w in mats:
+            q4.q4_gemv(w, xs[shapes[name][1]], y=ys[name])
+
+    # eager warm-up (loads modules, sets kernel attributes), then capture
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    assert q4.q4_sync_status() == q4.Q4_OK
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+        step()
+    torch.cuda.synchronize()
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ms = time_region(torch, graph.replay, args.steps, args.warmup, stream)
+    if world > 1:
+        dist.barrier()
+    st = q4.q4_sync_status()
+    assert st == q4.Q4_OK, q4.status_string(st)
+    ms_eager = time_region(torch, step, max(3, args.steps // 10), 2, stream)
+    ms_eager /= max(3, args.steps // 10)
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    value = world * step_bytes * args.steps / (ms_max * 1e-3) / 1e9
+
+    # ---- bf16 reference on one layer of the same shapes (436 MB > L2)
+    bf_mats = []
+    for name, (out, inn) in shapes.items():
+        bf_mats.append((name, wl.normal_weight(out, inn, 10, device=device).to(torch.bfloat16)))
+    bf_bytes = sum(dense_bytes(*shapes[n], B) for n, _ in bf_mats)
+
+    def bf_step():
+        for name, Wb in bf_mats:
+            q4.bf16_gemv_ref_bw(Wb, xs[shapes[name][1]], y=ys[name])
+
+    for _ in range(3):
+        bf_step()
+    torch.cuda.synchronize()
+    bgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(bgraph, capture_error_mode="thread_local"):
+        bf_step()
+    nbf = max(20, args.steps // 4)
+    ms_bf = time_region(torch, bgraph.replay, nbf, 3, stream) / nbf
+    int4_layer_ms = ms_per_step / layers
+    del bf_mats, bgraph
+
+    # ---- quantize + pack throughput on one layer (fp16 in, codes out)
+    qW = [(n, wl.normal_weight(*shapes[n], 11, device=device)) for n in shapes]
+    qbytes = sum(quant_bytes(*shapes[n], 128) for n, _ in qW)
+    qouts = [(torch.empty(o, i // 2, dtype=torch.uint8, device=device),
+              torch.empty(o, i // 128, dtype=torch.float16, device=device)) for o, i in shapes.values()]
+
+    def q_step():
+        for (n, W), (qo, so) in zip(qW, qouts):
+            q4.q4_quantize_pack(W, 128, True, qweight=qo, scales=so)
+
+    nq = max(10, args.steps // 20)
+    ms_q = time_region(torch, q_step, nq, 2, stream) / nq
+    del qW, qouts
+
+    # ---- end to end through the public API with host buffers
+    x_host = {k: v.cpu().pin_memory() for k, v in xs.items()}
+    y_host = torch.empty(B, shapes["down_proj"][0], dtype=torch.bfloat16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in x_host.values())
+    d2h = y_host.numel() * y_host.element_size()
+    last = ys["down_proj"]
+
+    def e2e_step():
+        for k, v in x_host.items():
+            xs[k].copy_(v, non_blocking=True)
+        graph.replay()
+        y_host.copy_(last, non_blocking=True)
+        stream.synchronize()
+
+    ne = max(10, args.steps // 10)
+    for _ in range(2):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(ne):
+        e2e_step()
+    e2e_s = torch.tensor([time.perf_counter() - t0], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(e2e_s, op=dist.ReduceOp.MAX)
+    e2e_value = world * step_bytes * ne / float(e2e_s.item()) / 1e9
+
+    clocks = clk.summary()
+    peak = peaks["hbm_gbs"]
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02^2) fp16 weights quantized on device; bf16 N(0,1) activations)",
+        "config": {"workload": f"Llama-3-8B decode linears q,k,v,o,gate,up,down x {layers} distinct layers per step",
+                   "batch": B, "group_size": 128, "symmetric": True, "layers": layers,
+                   "linears_per_step": launches_per_step,
+                   "bytes_per_step": step_bytes, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB of packed weights per step, 126 MB L2)",
+                   "timing": "CUDA graph of the step, CUDA events on the launching stream"},
+        "us_per_layer": round(int4_layer_ms * 1e3, 3),
+        "pct_of_8TBs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+        "pct_of_measured_hbm": round(100 * value / world / peak, 2),
+        "eager_us_per_layer": round(ms_eager / layers * 1e3, 3),
+        "bf16": {"us_per_layer": round(ms_bf * 1e3, 3),
+                 "gbs": round(bf_bytes / (ms_bf * 1e-3) / 1e9, 1),
+                 "speedup_int4_vs_bf16_B1": round(ms_bf / int4_layer_ms, 3)},
+        "quantize_pack": {"gbs": round(qbytes / (ms_q * 1e-3) / 1e9, 1),
+                          "us_per_layer": round(ms_q * 1e3, 2)},
+        "roofline": {"bound": "hbm", "achieved": round(value / world, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(value / world / peak, 4),
+                     "peak_kind": peak_kind, "traffic": None,
+                     "kernel": "q4_gemv_kernel<bf16,g128,sym>",
+                     "bytes_per_launch_avg": step_bytes // launches_per_step},
+        "clocks": clocks,
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": ne},
+        "gpu_launches": args.steps * launches_per_step,
+    }
+    if rank == 0:
+        out["cpu_baseline"] = cpu_baseline() if (world == 1 and not args.no_cpu_baseline) else None
+        print(json.dumps(out), flush=True)
+    del graph
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------- CPU oracle timing
+def _oracle_layer():
+    """One Llama-3-8B layer (7 linears, sym g128) quantized by the CPU oracle,
+    with its B=1 activations.  Preparation is not timed."""
+    import numpy as np
+    import oracle
+    from post_weight_quantization_group_b200 import workloads as wl
+
+    oracle.build()
+    prepared = []
+    for name, (out, inn) in wl.LLAMA3_8B.items():
+        W = wl.normal_weight(out, inn, wl.llama3_8b_layer_seeds(0)[name]).float().numpy()
+        q, s, _ = oracle.quantize_pack(W, 128, True)
+        x = wl.activations(1, inn, 17 + inn).float().numpy().astype(np.float64)
+        prepared.append((out, inn, q, s, x))
+    return prepared
+
+
+def _oracle_pass(prepared, frac=1.0):
+    """fp64 oracle product over the first ceil(frac * out) rows of each linear;
+    returns algorithmic bytes processed."""
+    import numpy as np
+    import oracle
+    nbytes = 0
+    for out, inn, q, s, x in prepared:
+        n = max(1, min(out, int(round(out * frac))))
+        rows = np.arange(n, dtype=np.int64)
+        oracle.gemv(q, s, None, out, inn, 128, True, x, rows=rows)
+        nbytes += algo_bytes(n, inn, 128, 1)
+    return nbytes
+
+
+def cpu_baseline():
+    prepared = _oracle_layer()
+    t0 = time.perf_counter()
+    nbytes = 0
+    for _ in range(3):
+        nbytes += _oracle_pass(prepared)
+    dt = time.perf_counter() - t0
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "3 passes over 1 of 32 Llama-3-8B layers (7 linears, sym g128, B=1), "
+                      "fp64 product of the CPU oracle, single thread",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    prepared = _oracle_layer()
+    # calibrate, then size each step's row sample so the run takes ~90 s
+    t0 = time.perf_counter()
+    cb = _oracle_pass(prepared, 0.02)
+    rate = cb / (time.perf_counter() - t0)
+    layer_bytes = sum(algo_bytes(o, i, 128, 1) for o, i, *_ in prepared)
+    frac = min(1.0, max(1e-4, 90.0 * rate / (args.steps + args.warmup) / layer_bytes))
+    for _ in range(args.warmup):
+        _oracle_pass(prepared, frac)
+    t0 = time.perf_counter()
+    nbytes = 0
+    for _ in range(args.steps):
+        nbytes += _oracle_pass(prepared, frac)
+    dt = time.perf_counter() - t0
+    value = nbytes / dt / 1e9
+    sample = (f"per step: the first {100 * frac:.3g}% of the rows of each of the 7 linears of "
+              f"one Llama-3-8B layer (sym g128, B=1), fp64 product, single thread")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,0.02^2) fp16 weights, bf16 N(0,1) activations)",
+        "config": {"workload": "Llama-3-8B decode linears q,k,v,o,gate,up,down, B=1, sym g128 "
+                               "(CPU oracle on a row sample)", "batch": 1, "group_size": 128},
+        "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama3-8b", choices=["llama3-8b"])
+    ap.add_argument("--layers", type=int, default=32,
+                    help="distinct decoder layers per step (32 = the Llama-3-8B depth)")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip timing the CPU oracle (profiling runs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

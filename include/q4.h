@@ -1,0 +1,190 @@
+/*
+ * q4.h -- C ABI of the group-wise INT4 weight quantization and W4A16 decode
+ * library for NVIDIA B200 (sm_100a).
+ *
+ * The operations are those of the pages this library follows:
+ *
+ *   affine quantization  q = clamp(round(w / s) + z, qmin, qmax),
+ *   dequantization       w_hat = s * (q - z),
+ *     -- "LLM 后训练量化深度实战" (ybb.press), section 二, first equation;
+ *        arganzheng.life post-training-quantization-gptq-awq-and-rotation,
+ *        section 二.2 (基本形式与粒度);
+ *   symmetric scale s = max|w| / 7 (z = 0, codes in [-8, 7]) and asymmetric
+ *   scale s = (max - min) / 15 with integer zero point z (codes in [0, 15]),
+ *     -- arganzheng.life section 二.2; ybb.press section 二
+ *        (quantize_per_group: groups of group_size along in_features);
+ *   the decode product of W4A16: packed INT4 weights plus per-group scale /
+ *   zero are read from HBM, dequantised on chip and multiplied with 16-bit
+ *   activations, y = x W_hat^T,
+ *     -- arganzheng.life section 二.1 (decode GEMM [B, k] x [k, n]) and
+ *        section 二.3 (W4A16 dataflow: shift, mask, x s, + z on chip).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument is a DEVICE pointer (except `w`, the q4_weight
+ *    descriptor, which is a host struct passed by pointer and read during the
+ *    call only).  The caller owns all memory.  The library never allocates,
+ *    frees or synchronizes (except q4_sync_status) and enqueues all of its
+ *    work on `stream` (a cudaStream_t; NULL = the legacy default stream).
+ *  - Tensors are dense and row-major.  W and W_hat are [out, in]; x is
+ *    [B, in]; y is [B, out]; scales and zeros are [out, in / group_size].
+ *  - Packed codes: qweight is [out, in / 2] bytes; byte j of a row holds
+ *    element 2j in its low nibble and element 2j+1 in its high nibble.
+ *    Symmetric codes are stored as 4-bit two's complement (q & 0xF);
+ *    asymmetric codes as unsigned 4-bit integers.
+ *  - Scales are fp16.  Zero points are fp16 holding integers in [0, 15];
+ *    zeros == NULL if and only if symmetric.
+ *  - Argument errors are returned synchronously and nothing is launched.
+ *    Errors that happen on the device after a successful return (a bounded
+ *    wait that ran out) are reported by q4_sync_status.  A CUDA launch error
+ *    is returned as Q4_ERR_CUDA.
+ *  - Weights or activations holding Inf / NaN give unspecified values but no
+ *    fault.
+ */
+#ifndef Q4_H
+#define Q4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define Q4_API __attribute__((visibility("default")))
+#else
+#define Q4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    Q4_OK = 0,
+    Q4_ERR_INVALID_ARG = 1,  /* NULL pointer, bad enum value, negative size */
+    Q4_ERR_SHAPE = 2,        /* group_size does not divide in, odd sizes, B out of range */
+    Q4_ERR_ALIGNMENT = 3,    /* a pointer is not aligned as the call requires */
+    Q4_ERR_UNSUPPORTED = 4,  /* bits != 4, a group size or dtype this call does not take */
+    Q4_ERR_CUDA = 5,         /* a CUDA runtime or launch error */
+    Q4_ERR_TIMEOUT = 6       /* a kernel's bounded wait ran out (see q4_sync_status) */
+} q4_status;
+
+typedef enum { Q4_F16 = 0, Q4_BF16 = 1, Q4_F32 = 2 } q4_dtype;
+
+/* A cudaStream_t, passed as an opaque pointer so that this header needs no
+ * CUDA include. */
+typedef void* q4_stream;
+
+/* A quantized weight matrix, as q4_quantize_pack writes it. */
+typedef struct q4_weight {
+    const uint8_t* qweight;  /* [out, in/2] packed codes, 16-byte aligned */
+    const void* scales;      /* [out, in/group_size] fp16, 2-byte aligned */
+    const void* zeros;       /* [out, in/group_size] fp16 integers, NULL iff symmetric */
+    int64_t out;             /* rows (output features), >= 0 */
+    int64_t in;              /* columns (input features, the reduction dim), > 0 */
+    int32_t group_size;      /* codes sharing one scale along `in` */
+    int32_t bits;            /* must be 4 */
+    int32_t symmetric;       /* 1: codes in [-8, 7], z = 0;  0: codes in [0, 15] */
+} q4_weight;
+
+/*
+ * Group-wise INT4 round-to-nearest quantization and packing of W [out, in].
+ *
+ * For each row r and group j (elements k in [j*g, (j+1)*g)), in fp32:
+ *   symmetric:  s = fp16(max|w| / 7);          q = clamp(rne(w / s), -8, 7)
+ *   asymmetric: s = fp16((max - min) / 15);   z = clamp(rne(-min / s), 0, 15)
+ *               q = clamp(rne(w / s) + z, 0, 15)
+ * where rne rounds half to even, the divisions are IEEE fp32 divisions, and
+ * the stored fp16 scale is the one used to compute the codes.  A group whose
+ * stored scale is 0 gets codes 0 (and z = 0).  (Sources: ybb.press section
+ * 二 quantize_per_group; arganzheng.life section 二.2; "压缩算法"
+ * (cs-knowledge-wiki) section 7.4.1.2, pack_int4.)
+ *
+ *   W          [out, in] fp16 or bf16 (w_dtype), 16-byte aligned
+ *   group_size even, divides `in`; any even value is accepted
+ *   bits       must be 4, else Q4_ERR_UNSUPPORTED
+ *   qweight    [out, in/2] output, 4-byte aligned
+ *   scales     [out, in/group_size] fp16 output, 2-byte aligned
+ *   zeros      [out, in/group_size] fp16 output; NULL iff symmetric
+ * `in` must be a multiple of 8.  Results are bit-identical to the CPU oracle.
+ */
+Q4_API q4_status q4_quantize_pack(const void* W, q4_dtype w_dtype, int64_t out, int64_t in,
+                           int32_t group_size, int32_t bits, int32_t symmetric,
+                           uint8_t* qweight, void* scales, void* zeros, q4_stream stream);
+
+/*
+ * Dequantization W_hat = s * (q - z), [out, in], in fp16, bf16 or fp32.
+ * s * (q - z) is exact in fp32; fp16 / bf16 outputs are that value rounded
+ * to nearest even.  (ybb.press section 二; arganzheng.life section 二.2.)
+ * Any even group size dividing `in`; `in` a multiple of 8; W_hat 16-byte
+ * aligned.
+ */
+Q4_API q4_status q4_dequant(const q4_weight* w, void* W_hat, q4_dtype out_dtype, q4_stream stream);
+
+/*
+ * Fused W4A16 decode product for small batches:
+ *   y[b, r] = sum_k x[b, k] * s[r, k/g] * (q[r, k] - z[r, k/g]),   1 <= B <= 8.
+ * The packed weights are streamed from HBM once; codes are unpacked to exact
+ * 16-bit integers in registers, multiplied with x on the tensor cores with
+ * fp32 accumulation per group, and each group's partial sum is scaled by its
+ * fp32 scale (arganzheng.life section 二.2: per-group scales must be applied
+ * inside the K accumulation; section 二.3: on-chip dequantization).
+ *
+ *   x      [B, in] bf16 or fp16 (x_dtype), 16-byte aligned
+ *   y      [B, out] in y_dtype (= x_dtype or Q4_F32), 16-byte aligned
+ *   group_size 32, 64 or 128 (else Q4_ERR_UNSUPPORTED); `in` a multiple of 32
+ *   qweight 16-byte aligned.
+ * Summation order differs from the fp64 oracle; results agree within
+ * |y - y_ref| <= 4e-3 * (|y_ref| + rms(y_ref)) (the bf16 output rounding
+ * included).
+ */
+Q4_API q4_status q4_gemv(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B, void* y,
+                  q4_dtype y_dtype, q4_stream stream);
+
+/*
+ * The same product for batches 1 <= B <= 128 (the skinny-GEMM regime of
+ * arganzheng.life section 二.4, where W4A16 turns compute-bound near
+ * B = ridge / 4).  B <= 8 runs the q4_gemv kernel.  Same arguments and
+ * requirements as q4_gemv.
+ */
+Q4_API q4_status q4_gemm_skinny(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B,
+                         void* y, q4_dtype y_dtype, q4_stream stream);
+
+/*
+ * The unquantised bf16 product y = x W^T with fp32 accumulation, the
+ * baseline the INT4 path is compared against and the probe of the bandwidth
+ * a weight stream reaches (ybb.press section 一, roofline_bound; arganzheng.
+ * life section 二.4, BF16 vs W4A16 batch table).
+ *   W [out, in] bf16, x [B, in] bf16, y [B, out] bf16; 1 <= B <= 128;
+ *   `in` a multiple of 64; W, x, y 16-byte aligned.
+ */
+Q4_API q4_status bf16_gemv_ref_bw(const void* W, int64_t out, int64_t in, const void* x, int64_t B,
+                           void* y, q4_stream stream);
+
+/*
+ * Waits for `stream`, then reports the first device-side error recorded
+ * since the previous call (Q4_ERR_TIMEOUT when a kernel's bounded wait ran
+ * out) or a pending CUDA error (Q4_ERR_CUDA), and clears the record.
+ */
+Q4_API q4_status q4_sync_status(q4_stream stream);
+
+/*
+ * Self-test of the bounded-wait machinery every pipelined kernel uses: one
+ * CTA waits on a shared-memory barrier that nothing ever arrives on, gives up
+ * after limit_ns nanoseconds (1 <= limit_ns <= 1e9, else Q4_ERR_INVALID_ARG)
+ * and records the timeout; a following q4_sync_status returns
+ * Q4_ERR_TIMEOUT and clears it.  No memory is touched, nothing faults, and
+ * the context stays usable.  (The pages have no counterpart; this checks the
+ * library's failure path without a GPU fault.)
+ */
+Q4_API q4_status q4_selftest_wait_timeout(int64_t limit_ns, q4_stream stream);
+
+/* Human-readable name of a status code (static storage). */
+Q4_API const char* q4_status_string(q4_status s);
+
+/* Library version string (static storage). */
+Q4_API const char* q4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4_H */

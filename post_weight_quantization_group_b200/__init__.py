@@ -1,0 +1,234 @@
+"""Python binding of the q4 C ABI (include/q4.h) for NVIDIA B200.
+
+Argument marshalling only: every step of the quantize / dequantize / decode
+product path runs in the CUDA kernels of ``libq4.so``.  PyTorch provides the
+device memory (outputs are allocated here when not given) and the stream
+(``torch.cuda.current_stream()`` unless one is passed).  There is no CPU path:
+if ``libq4.so`` cannot be loaded every call raises ``Q4LibraryError``.
+
+Names follow the C ABI: ``q4_quantize_pack``, ``q4_dequant``, ``q4_gemv``,
+``q4_gemm_skinny``, ``bf16_gemv_ref_bw``, ``q4_sync_status``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libq4.so")
+
+Q4_OK = 0
+Q4_ERR_INVALID_ARG = 1
+Q4_ERR_SHAPE = 2
+Q4_ERR_ALIGNMENT = 3
+Q4_ERR_UNSUPPORTED = 4
+Q4_ERR_CUDA = 5
+Q4_ERR_TIMEOUT = 6
+
+Q4_F16, Q4_BF16, Q4_F32 = 0, 1, 2
+_DT = {torch.float16: Q4_F16, torch.bfloat16: Q4_BF16, torch.float32: Q4_F32}
+
+# every symbol include/q4.h declares
+ABI_SYMBOLS = (
+    "q4_quantize_pack", "q4_dequant", "q4_gemv", "q4_gemm_skinny", "bf16_gemv_ref_bw",
+    "q4_sync_status", "q4_status_string", "q4_version", "q4_selftest_wait_timeout",
+)
+
+
+class Q4LibraryError(RuntimeError):
+    """libq4.so is missing or failed to load (there is no fallback)."""
+
+
+class Q4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+class _CWeight(ctypes.Structure):
+    _fields_ = [
+        ("qweight", ctypes.c_void_p),
+        ("scales", ctypes.c_void_p),
+        ("zeros", ctypes.c_void_p),
+        ("out", ctypes.c_int64),
+        ("in_", ctypes.c_int64),
+        ("group_size", ctypes.c_int32),
+        ("bits", ctypes.c_int32),
+        ("symmetric", ctypes.c_int32),
+    ]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libq4.so (once) and declare the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise Q4LibraryError(
+            f"{path} not found: build it with `python -m post_weight_quantization_group_b200.build`")
+    try:
+        lib = ctypes.CDLL(path)
+    except OSError as e:  # pragma: no cover - environment dependent
+        raise Q4LibraryError(f"cannot load {path}: {e}") from e
+    P, I64, I32, S = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
+    W = ctypes.POINTER(_CWeight)
+    lib.q4_quantize_pack.argtypes = [P, S, I64, I64, I32, I32, I32, P, P, P, P]
+    lib.q4_dequant.argtypes = [W, P, S, P]
+    lib.q4_gemv.argtypes = [W, P, S, I64, P, S, P]
+    lib.q4_gemm_skinny.argtypes = [W, P, S, I64, P, S, P]
+    lib.bf16_gemv_ref_bw.argtypes = [P, I64, I64, P, I64, P, P]
+    lib.q4_sync_status.argtypes = [P]
+    lib.q4_selftest_wait_timeout.argtypes = [I64, P]
+    for f in ("q4_quantize_pack", "q4_dequant", "q4_gemv", "q4_gemm_skinny",
+              "bf16_gemv_ref_bw", "q4_sync_status", "q4_selftest_wait_timeout"):
+        getattr(lib, f).restype = S
+    lib.q4_status_string.argtypes = [S]
+    lib.q4_status_string.restype = ctypes.c_char_p
+    lib.q4_version.argtypes = []
+    lib.q4_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().q4_status_string(int(status)).decode()
+
+
+def version() -> str:
+    return load_library().q4_version().decode()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("q4 takes device tensors only")
+    if not t.is_contiguous():
+        raise ValueError("q4 takes contiguous tensors only")
+    return t.data_ptr()
+
+
+def _check(status: int, what: str):
+    if status != Q4_OK:
+        raise Q4Error(status, what)
+
+
+@dataclass
+class Q4Weight:
+    """A packed INT4 weight: codes [out, in/2] uint8, fp16 scales [out, in/g],
+    fp16 zero points [out, in/g] (None if symmetric)."""
+    qweight: torch.Tensor
+    scales: torch.Tensor
+    zeros: torch.Tensor | None
+    out: int
+    in_features: int
+    group_size: int
+    symmetric: bool
+    bits: int = 4
+
+    def c_struct(self) -> _CWeight:
+        return _CWeight(_ptr(self.qweight), _ptr(self.scales), _ptr(self.zeros), self.out,
+                        self.in_features, self.group_size, self.bits, int(self.symmetric))
+
+    @property
+    def nbytes(self) -> int:
+        n = self.qweight.numel() + self.scales.numel() * 2
+        return n + (self.zeros.numel() * 2 if self.zeros is not None else 0)
+
+
+def q4_quantize_pack(W: torch.Tensor, group_size: int = 128, symmetric: bool = True,
+                     bits: int = 4, qweight: torch.Tensor | None = None,
+                     scales: torch.Tensor | None = None, zeros: torch.Tensor | None = None,
+                     stream=None) -> Q4Weight:
+    lib = load_library()
+    if W.dim() != 2 or W.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("W must be a 2-D fp16 or bf16 tensor")
+    out, inn = W.shape
+    G = inn // group_size if group_size > 0 else 0
+    dev = W.device
+    if qweight is None:
+        qweight = torch.empty(out, inn // 2, dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(out, G, dtype=torch.float16, device=dev)
+    if zeros is None and not symmetric:
+        zeros = torch.empty(out, G, dtype=torch.float16, device=dev)
+    st = lib.q4_quantize_pack(_ptr(W), _DT[W.dtype], out, inn, group_size, bits,
+                              int(symmetric), _ptr(qweight), _ptr(scales), _ptr(zeros),
+                              _stream(stream))
+    _check(st, "q4_quantize_pack")
+    return Q4Weight(qweight, scales, zeros, out, inn, group_size, bool(symmetric), bits)
+
+
+def q4_dequant(w: Q4Weight, out_dtype=torch.float32, W_hat: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    lib = load_library()
+    if W_hat is None:
+        W_hat = torch.empty(w.out, w.in_features, dtype=out_dtype, device=w.qweight.device)
+    cw = w.c_struct()
+    st = lib.q4_dequant(ctypes.byref(cw), _ptr(W_hat), _DT[W_hat.dtype], _stream(stream))
+    _check(st, "q4_dequant")
+    return W_hat
+
+
+def _product(fn_name: str, w: Q4Weight, x: torch.Tensor, y, y_dtype, stream):
+    lib = load_library()
+    if x.dim() != 2:
+        raise ValueError("x must be [B, in]")
+    B = x.shape[0]
+    if y is None:
+        y = torch.empty(B, w.out, dtype=y_dtype or x.dtype, device=x.device)
+    cw = w.c_struct()
+    st = getattr(lib, fn_name)(ctypes.byref(cw), _ptr(x), _DT[x.dtype], B, _ptr(y),
+                               _DT[y.dtype], _stream(stream))
+    _check(st, fn_name)
+    return y
+
+
+def q4_gemv(w: Q4Weight, x: torch.Tensor, y: torch.Tensor | None = None, y_dtype=None,
+            stream=None) -> torch.Tensor:
+    """y = x W_hat^T for B <= 8 (x [B, in] bf16/fp16; y [B, out] x.dtype or fp32)."""
+    return _product("q4_gemv", w, x, y, y_dtype, stream)
+
+
+def q4_gemm_skinny(w: Q4Weight, x: torch.Tensor, y: torch.Tensor | None = None, y_dtype=None,
+                   stream=None) -> torch.Tensor:
+    """y = x W_hat^T for B <= 128."""
+    return _product("q4_gemm_skinny", w, x, y, y_dtype, stream)
+
+
+def bf16_gemv_ref_bw(W: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """y = x W^T for bf16 W [out, in], x [B, in], B <= 128."""
+    lib = load_library()
+    out, inn = W.shape
+    B = x.shape[0]
+    if y is None:
+        y = torch.empty(B, out, dtype=torch.bfloat16, device=x.device)
+    st = lib.bf16_gemv_ref_bw(_ptr(W), out, inn, _ptr(x), B, _ptr(y), _stream(stream))
+    _check(st, "bf16_gemv_ref_bw")
+    return y
+
+
+def q4_sync_status(stream=None) -> int:
+    """Synchronize ``stream`` and return (and clear) the device status."""
+    return load_library().q4_sync_status(_stream(stream))
+
+
+def q4_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
+    """Launch a kernel whose bounded wait can never be satisfied; returns the
+    launch status (the timeout is then reported by q4_sync_status)."""
+    return load_library().q4_selftest_wait_timeout(int(limit_ns), _stream(stream))

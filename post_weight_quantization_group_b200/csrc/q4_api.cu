@@ -1,0 +1,453 @@
+// q4_api.cu -- the C ABI of include/q4.h: argument validation, launch
+// planning, TMA descriptor encoding and kernel launches.  All kernels live in
+// this translation unit (q4_quant.cuh, q4_gemv.cuh, q4_skinny.cuh).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <utility>
+
+#include "q4.h"
+#include "q4_device.cuh"
+#include "q4_gemv.cuh"
+#include "q4_quant.cuh"
+
+namespace {
+
+using namespace q4dev;
+
+// Device-side error word (see q4dev::kStatusTimeout); read and cleared by
+// q4_sync_status.
+__device__ unsigned g_q4_status;
+
+// --------------------------------------------------------------- helpers
+constexpr int kMaxDevices = 64;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int current_device() {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess) return -1;
+    return d;
+}
+
+int sm_count(int dev) {
+    static std::atomic<int> cache[kMaxDevices];
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+int max_smem_optin(int dev) {
+    static std::atomic<int> cache[kMaxDevices];
+    if (dev < 0 || dev >= kMaxDevices) return 227 * 1024;
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        n <= 0)
+        n = 227 * 1024;
+    cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda
+// link dependency).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `elem` bytes, box [box_rows, box_cols],
+// 128-byte swizzle, out-of-bounds elements read as zero.
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem,
+                  uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem)};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+q4_status launch_status(cudaError_t e) {
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return e == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+}
+
+// Per-(kernel, device) one-time attribute setup.
+template <typename K>
+bool set_kernel_attrs(K kernel, int smem_bytes, bool nonportable_cluster) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem_bytes);
+    if (e != cudaSuccess) return false;
+    if (nonportable_cluster) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return false;
+    }
+    return true;
+}
+
+// Split-K plan for the streaming kernels: rows per CTA `rt`, `nchunks` chunks
+// of K.  S CTAs of one cluster share a row tile; aim for >= 2 CTAs per SM.
+struct SplitPlan {
+    int S, cps;
+};
+
+SplitPlan plan_split(int64_t out, int nchunks, int rt, int sms) {
+    const int64_t row_tiles = (out + rt - 1) / rt;
+    int S = 1;
+    while (S < 8 && row_tiles * S < 2LL * sms && nchunks >= 2 * S) S *= 2;
+    int cps = (nchunks + S - 1) / S;
+    S = (nchunks + cps - 1) / cps;
+    return {S, cps};
+}
+
+template <typename... KArgs, typename... Args>
+q4_status launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                         int cluster_x, cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (cluster_x > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cluster_x;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return launch_status(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
+}
+
+bool valid_dtype(int d) { return d == Q4_F16 || d == Q4_BF16 || d == Q4_F32; }
+
+q4_status validate_weight(const q4_weight* w) {
+    if (!w) return Q4_ERR_INVALID_ARG;
+    if (w->bits != 4) return Q4_ERR_UNSUPPORTED;
+    if (w->out < 0 || w->in <= 0 || w->group_size <= 0) return Q4_ERR_SHAPE;
+    if ((w->group_size & 1) || (w->in % w->group_size) != 0) return Q4_ERR_SHAPE;
+    if (w->symmetric != 0 && w->symmetric != 1) return Q4_ERR_INVALID_ARG;
+    if (w->out > 0 && (!w->qweight || !w->scales)) return Q4_ERR_INVALID_ARG;
+    if (w->out > 0 && !w->symmetric && !w->zeros) return Q4_ERR_INVALID_ARG;
+    if (w->symmetric && w->zeros) return Q4_ERR_INVALID_ARG;
+    if (!aligned(w->scales, 2) || (w->zeros && !aligned(w->zeros, 2))) return Q4_ERR_ALIGNMENT;
+    return Q4_OK;
+}
+
+// A wait that can never be satisfied, bounded by limit_ns.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbarrier_init_cluster();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, &g_q4_status, limit_ns);
+}
+
+// --------------------------------------------------------- quantize_pack
+template <bool SYM, bool BF16IN>
+q4_status run_quantize(const void* W, int64_t out, int64_t in, int g, uint8_t* qweight,
+                       __half* scales, __half* zeros, cudaStream_t st) {
+    const int dev = current_device();
+    const int sms = sm_count(dev);
+    const int64_t ngroups = out * (in / g);
+    if (ngroups == 0) return Q4_OK;
+    const bool fast = (g == 8 || g == 16 || g == 32 || g == 64 || g == 128 || g == 256) &&
+                      aligned(qweight, 4);
+    if (fast) {
+        const int64_t nchunks = out * in / 8;
+        const int64_t want = (nchunks + 255) / 256;
+        const int blocks = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
+        uint32_t* qw = reinterpret_cast<uint32_t*>(qweight);
+        switch (g) {
+#define Q4_QCASE(GV)                                                                              \
+    case GV:                                                                                      \
+        quantize_pack_kernel<GV, SYM, BF16IN><<<blocks, 256, 0, st>>>(W, nchunks, qw, scales, zeros); \
+        break;
+            Q4_QCASE(8) Q4_QCASE(16) Q4_QCASE(32) Q4_QCASE(64) Q4_QCASE(128) Q4_QCASE(256)
+#undef Q4_QCASE
+        }
+        return launch_status(cudaSuccess);
+    }
+    const int64_t want = (ngroups * 32 + 255) / 256;
+    const int blocks = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
+    quantize_pack_generic_kernel<SYM, BF16IN><<<blocks, 256, 0, st>>>(W, ngroups, g, qweight,
+                                                                      scales, zeros);
+    return launch_status(cudaSuccess);
+}
+
+// ------------------------------------------------------------------ GEMV
+constexpr int kGemvMT = 2;
+constexpr int kGemvCW = 4;
+constexpr int kGemvStages = 4;
+constexpr int kGemvRT = kGemvCW * kGemvMT * 16;
+
+template <bool BF16, int GS, bool SYM>
+q4_status run_gemv(const q4_weight* w, const void* x, int64_t B, void* y, int ydt,
+                   cudaStream_t st) {
+    const int dev = current_device();
+    const int sms = sm_count(dev);
+    const int nchunks = static_cast<int>((w->in + kChunkCodes - 1) / kChunkCodes);
+    SplitPlan p = plan_split(w->out, nchunks, kGemvRT, sms);
+    GemvGeom geo = gemv_geom(kGemvRT, kGemvStages, p.cps, static_cast<int>(B), GS, SYM);
+    const int smax = max_smem_optin(dev);
+    while (geo.total > static_cast<size_t>(smax) && p.S < 16) {
+        p.S = p.S * 2 > 16 ? 16 : p.S * 2;
+        p.cps = (nchunks + p.S - 1) / p.S;
+        p.S = (nchunks + p.cps - 1) / p.cps;
+        geo = gemv_geom(kGemvRT, kGemvStages, p.cps, static_cast<int>(B), GS, SYM);
+        if (p.S == 16 || p.cps == 1) break;
+    }
+    if (geo.total > static_cast<size_t>(smax)) return Q4_ERR_UNSUPPORTED;
+
+    CUtensorMap tmap;
+    if (!make_tmap_2d(&tmap, w->qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                      static_cast<uint64_t>(w->out), static_cast<uint64_t>(w->in / 2),
+                      kGemvRT, kChunkBytes))
+        return Q4_ERR_CUDA;
+    auto kernel = q4_gemv_kernel<BF16, GS, SYM, kGemvMT, kGemvCW, kGemvStages>;
+    if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), p.S > 8)) return Q4_ERR_CUDA;
+    unsigned* status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
+        return Q4_ERR_CUDA;
+    const dim3 grid(p.S, static_cast<unsigned>((w->out + kGemvRT - 1) / kGemvRT));
+    return launch_cluster(kernel, grid, dim3((kGemvCW + 1) * 32), geo.total, p.S, st, tmap,
+                          reinterpret_cast<const __half*>(w->scales),
+                          reinterpret_cast<const __half*>(w->zeros),
+                          reinterpret_cast<const uint16_t*>(x), static_cast<int>(B), w->out,
+                          w->in, p.cps, nchunks, y, ydt, status);
+}
+
+template <bool BF16>
+q4_status dispatch_gemv(const q4_weight* w, const void* x, int64_t B, void* y, int ydt,
+                        cudaStream_t st) {
+    const bool sym = w->symmetric != 0;
+    switch (w->group_size) {
+        case 32: return sym ? run_gemv<BF16, 32, true>(w, x, B, y, ydt, st)
+                            : run_gemv<BF16, 32, false>(w, x, B, y, ydt, st);
+        case 64: return sym ? run_gemv<BF16, 64, true>(w, x, B, y, ydt, st)
+                            : run_gemv<BF16, 64, false>(w, x, B, y, ydt, st);
+        case 128: return sym ? run_gemv<BF16, 128, true>(w, x, B, y, ydt, st)
+                             : run_gemv<BF16, 128, false>(w, x, B, y, ydt, st);
+        default: return Q4_ERR_UNSUPPORTED;
+    }
+}
+
+q4_status validate_product(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B,
+                           void* y, q4_dtype y_dtype, int64_t bmax) {
+    q4_status s = validate_weight(w);
+    if (s != Q4_OK) return s;
+    if (!valid_dtype(x_dtype) || !valid_dtype(y_dtype)) return Q4_ERR_INVALID_ARG;
+    if (x_dtype == Q4_F32) return Q4_ERR_UNSUPPORTED;
+    if (y_dtype != x_dtype && y_dtype != Q4_F32) return Q4_ERR_UNSUPPORTED;
+    if (B < 1 || B > bmax) return Q4_ERR_SHAPE;
+    if (w->group_size != 32 && w->group_size != 64 && w->group_size != 128)
+        return Q4_ERR_UNSUPPORTED;
+    if ((w->in % 32) != 0) return Q4_ERR_SHAPE;
+    if (w->in > (int64_t(1) << 30) || w->out > int64_t(65535) * 128) return Q4_ERR_SHAPE;
+    if (w->out == 0) return Q4_OK;  // nothing to read or write
+    if (!x || !y) return Q4_ERR_INVALID_ARG;
+    if (!aligned(w->qweight, 16) || !aligned(x, 16) || !aligned(y, 16)) return Q4_ERR_ALIGNMENT;
+    return Q4_OK;
+}
+
+}  // namespace
+
+// ======================================================================= ABI
+extern "C" {
+
+const char* q4_version(void) { return "q4-b200 0.1 (sm_100a)"; }
+
+const char* q4_status_string(q4_status s) {
+    switch (s) {
+        case Q4_OK: return "Q4_OK";
+        case Q4_ERR_INVALID_ARG: return "Q4_ERR_INVALID_ARG";
+        case Q4_ERR_SHAPE: return "Q4_ERR_SHAPE";
+        case Q4_ERR_ALIGNMENT: return "Q4_ERR_ALIGNMENT";
+        case Q4_ERR_UNSUPPORTED: return "Q4_ERR_UNSUPPORTED";
+        case Q4_ERR_CUDA: return "Q4_ERR_CUDA";
+        case Q4_ERR_TIMEOUT: return "Q4_ERR_TIMEOUT";
+    }
+    return "Q4_ERR_UNKNOWN";
+}
+
+q4_status q4_quantize_pack(const void* W, q4_dtype w_dtype, int64_t out, int64_t in,
+                           int32_t group_size, int32_t bits, int32_t symmetric, uint8_t* qweight,
+                           void* scales, void* zeros, q4_stream stream) {
+    if (w_dtype != Q4_F16 && w_dtype != Q4_BF16) {
+        return valid_dtype(w_dtype) ? Q4_ERR_UNSUPPORTED : Q4_ERR_INVALID_ARG;
+    }
+    if (bits != 4) return Q4_ERR_UNSUPPORTED;
+    if (symmetric != 0 && symmetric != 1) return Q4_ERR_INVALID_ARG;
+    if (out < 0 || in <= 0 || group_size <= 0) return Q4_ERR_SHAPE;
+    if ((group_size & 1) || (in % group_size) != 0 || (in % 8) != 0) return Q4_ERR_SHAPE;
+    if (out == 0) return Q4_OK;
+    if (!W || !qweight || !scales) return Q4_ERR_INVALID_ARG;
+    if (symmetric ? (zeros != nullptr) : (zeros == nullptr)) return Q4_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(qweight, 4) || !aligned(scales, 2) ||
+        (zeros && !aligned(zeros, 2)))
+        return Q4_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    __half* s = reinterpret_cast<__half*>(scales);
+    __half* z = reinterpret_cast<__half*>(zeros);
+    const bool bf = (w_dtype == Q4_BF16);
+    if (symmetric)
+        return bf ? run_quantize<true, true>(W, out, in, group_size, qweight, s, z, st)
+                  : run_quantize<true, false>(W, out, in, group_size, qweight, s, z, st);
+    return bf ? run_quantize<false, true>(W, out, in, group_size, qweight, s, z, st)
+              : run_quantize<false, false>(W, out, in, group_size, qweight, s, z, st);
+}
+
+q4_status q4_dequant(const q4_weight* w, void* W_hat, q4_dtype out_dtype, q4_stream stream) {
+    q4_status s = validate_weight(w);
+    if (s != Q4_OK) return s;
+    if (!valid_dtype(out_dtype)) return Q4_ERR_INVALID_ARG;
+    if ((w->in % 8) != 0) return Q4_ERR_SHAPE;
+    if (w->out == 0) return Q4_OK;
+    if (!W_hat) return Q4_ERR_INVALID_ARG;
+    if (!aligned(W_hat, 16) || !aligned(w->qweight, 4)) return Q4_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int dev = current_device();
+    const int sms = sm_count(dev);
+    const int64_t nwords = w->out * w->in / 8;
+    const int64_t want = (nwords + 255) / 256;
+    const int blocks = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
+    const uint32_t* qw = reinterpret_cast<const uint32_t*>(w->qweight);
+    const __half* sc = reinterpret_cast<const __half*>(w->scales);
+    const __half* zc = reinterpret_cast<const __half*>(w->zeros);
+    const int g = w->group_size;
+    if (out_dtype == Q4_F32) {
+        if (w->symmetric)
+            dequant_kernel<float, true><<<blocks, 256, 0, st>>>(qw, sc, zc, nwords, w->in, g,
+                                                                reinterpret_cast<float*>(W_hat));
+        else
+            dequant_kernel<float, false><<<blocks, 256, 0, st>>>(qw, sc, zc, nwords, w->in, g,
+                                                                 reinterpret_cast<float*>(W_hat));
+    } else if (out_dtype == Q4_F16) {
+        if (w->symmetric)
+            dequant_kernel<__half, true><<<blocks, 256, 0, st>>>(qw, sc, zc, nwords, w->in, g,
+                                                                 reinterpret_cast<__half*>(W_hat));
+        else
+            dequant_kernel<__half, false><<<blocks, 256, 0, st>>>(qw, sc, zc, nwords, w->in, g,
+                                                                  reinterpret_cast<__half*>(W_hat));
+    } else {
+        if (w->symmetric)
+            dequant_kernel<__nv_bfloat16, true><<<blocks, 256, 0, st>>>(
+                qw, sc, zc, nwords, w->in, g, reinterpret_cast<__nv_bfloat16*>(W_hat));
+        else
+            dequant_kernel<__nv_bfloat16, false><<<blocks, 256, 0, st>>>(
+                qw, sc, zc, nwords, w->in, g, reinterpret_cast<__nv_bfloat16*>(W_hat));
+    }
+    return launch_status(cudaSuccess);
+}
+
+q4_status q4_gemv(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B, void* y,
+                  q4_dtype y_dtype, q4_stream stream) {
+    q4_status s = validate_product(w, x, x_dtype, B, y, y_dtype, 8);
+    if (s != Q4_OK) return s;
+    if (w->out == 0) return Q4_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int ydt = y_dtype == Q4_F32 ? 2 : (y_dtype == Q4_BF16 ? 1 : 0);
+    return x_dtype == Q4_BF16 ? dispatch_gemv<true>(w, x, B, y, ydt, st)
+                              : dispatch_gemv<false>(w, x, B, y, ydt, st);
+}
+
+q4_status q4_gemm_skinny(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B,
+                         void* y, q4_dtype y_dtype, q4_stream stream) {
+    q4_status s = validate_product(w, x, x_dtype, B, y, y_dtype, 128);
+    if (s != Q4_OK) return s;
+    if (B <= 8) return q4_gemv(w, x, x_dtype, B, y, y_dtype, stream);
+    return Q4_ERR_UNSUPPORTED;
+}
+
+q4_status bf16_gemv_ref_bw(const void* W, int64_t out, int64_t in, const void* x, int64_t B,
+                           void* y, q4_stream stream) {
+    if (out < 0 || in <= 0 || (in % 64) != 0) return Q4_ERR_SHAPE;
+    if (B < 1 || B > 128) return Q4_ERR_SHAPE;
+    if (in > (int64_t(1) << 30) || out > int64_t(65535) * 128) return Q4_ERR_SHAPE;
+    if (out == 0) return Q4_OK;
+    if (!W || !x || !y) return Q4_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(x, 16) || !aligned(y, 16)) return Q4_ERR_ALIGNMENT;
+    if (B > 8) return Q4_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int dev = current_device();
+    const int sms = sm_count(dev);
+    const int nchunks = static_cast<int>(in / kDenseChunkCols);
+    SplitPlan p = plan_split(out, nchunks, kGemvRT, sms);
+    DenseGeom geo = dense_geom(kGemvRT, kGemvStages, p.cps, static_cast<int>(B));
+    const int smax = max_smem_optin(dev);
+    while (geo.total > static_cast<size_t>(smax) && p.S < 16) {
+        p.S = p.S * 2 > 16 ? 16 : p.S * 2;
+        p.cps = (nchunks + p.S - 1) / p.S;
+        p.S = (nchunks + p.cps - 1) / p.cps;
+        geo = dense_geom(kGemvRT, kGemvStages, p.cps, static_cast<int>(B));
+        if (p.S == 16 || p.cps == 1) break;
+    }
+    if (geo.total > static_cast<size_t>(smax)) return Q4_ERR_UNSUPPORTED;
+    CUtensorMap tmap;
+    if (!make_tmap_2d(&tmap, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, static_cast<uint64_t>(out),
+                      static_cast<uint64_t>(in), kGemvRT, kDenseChunkCols))
+        return Q4_ERR_CUDA;
+    auto kernel = bf16_gemv_kernel<kGemvMT, kGemvCW, kGemvStages>;
+    if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), p.S > 8)) return Q4_ERR_CUDA;
+    unsigned* status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
+        return Q4_ERR_CUDA;
+    const dim3 grid(p.S, static_cast<unsigned>((out + kGemvRT - 1) / kGemvRT));
+    return launch_cluster(kernel, grid, dim3((kGemvCW + 1) * 32), geo.total, p.S, st, tmap,
+                          reinterpret_cast<const uint16_t*>(x), static_cast<int>(B), out, in,
+                          p.cps, nchunks, y, status);
+}
+
+q4_status q4_selftest_wait_timeout(int64_t limit_ns, q4_stream stream) {
+    if (limit_ns < 1 || limit_ns > 1000000000LL) return Q4_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint64_t>(limit_ns));
+    return launch_status(cudaSuccess);
+}
+
+q4_status q4_sync_status(q4_stream stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return Q4_ERR_CUDA;
+    unsigned h = 0;
+    if (cudaMemcpyFromSymbol(&h, g_q4_status, sizeof(h)) != cudaSuccess) return Q4_ERR_CUDA;
+    if (h != 0) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(g_q4_status, &zero, sizeof(zero)) != cudaSuccess)
+            return Q4_ERR_CUDA;
+        if (h & kStatusTimeout) return Q4_ERR_TIMEOUT;
+    }
+    return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+}
+
+}  // extern "C"
