@@ -64,7 +64,8 @@ typedef enum {
     Q4_ERR_ALIGNMENT = 3,    /* a pointer is not aligned as the call requires */
     Q4_ERR_UNSUPPORTED = 4,  /* bits != 4, a group size or dtype this call does not take */
     Q4_ERR_CUDA = 5,         /* a CUDA runtime or launch error */
-    Q4_ERR_TIMEOUT = 6       /* a kernel's bounded wait ran out (see q4_sync_status) */
+    Q4_ERR_TIMEOUT = 6,      /* a kernel's bounded wait ran out (see q4_sync_status) */
+    Q4_ERR_WORKSPACE = 7     /* workspace NULL or smaller than q4_workspace_bytes() */
 } q4_status;
 
 typedef enum { Q4_F16 = 0, Q4_BF16 = 1, Q4_F32 = 2 } q4_dtype;
@@ -120,6 +121,13 @@ Q4_API q4_status q4_quantize_pack(const void* W, q4_dtype w_dtype, int64_t out, 
 Q4_API q4_status q4_dequant(const q4_weight* w, void* W_hat, q4_dtype out_dtype, q4_stream stream);
 
 /*
+ * Bytes of device workspace that q4_gemv / q4_gemm_skinny need for a weight
+ * of this shape and a batch B, on the current device (an upper bound that
+ * depends on the device's SM count).  0 for invalid arguments.
+ */
+Q4_API size_t q4_workspace_bytes(int64_t out, int64_t in, int64_t B, int32_t group_size);
+
+/*
  * Fused W4A16 decode product for small batches:
  *   y[b, r] = sum_k x[b, k] * s[r, k/g] * (q[r, k] - z[r, k/g]),   1 <= B <= 8.
  * The packed weights are streamed from HBM once; codes are unpacked to exact
@@ -132,12 +140,23 @@ Q4_API q4_status q4_dequant(const q4_weight* w, void* W_hat, q4_dtype out_dtype,
  *   y      [B, out] in y_dtype (= x_dtype or Q4_F32), 16-byte aligned
  *   group_size 32, 64 or 128 (else Q4_ERR_UNSUPPORTED); `in` a multiple of 32
  *   qweight 16-byte aligned.
+ *   workspace  device scratch of at least q4_workspace_bytes(out, in, B,
+ *              group_size) bytes, 256-byte aligned, ZERO-FILLED before its
+ *              first use.  It holds per-row-tile counters, which every call
+ *              that completes leaves at zero, and partial sums, which need no
+ *              clearing; its layout is the same for every shape, so one
+ *              buffer (sized for the largest shape) serves any number of calls
+ *              of any shape in stream order.  Calls that may overlap on the
+ *              GPU need separate buffers.  After a call that ends in
+ *              Q4_ERR_TIMEOUT, re-zero it.
+ * The K reduction order is fixed, so results are bit-for-bit reproducible.
  * Summation order differs from the fp64 oracle; results agree within
  * |y - y_ref| <= 4e-3 * (|y_ref| + rms(y_ref)) (the bf16 output rounding
  * included).
  */
 Q4_API q4_status q4_gemv(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B, void* y,
-                  q4_dtype y_dtype, q4_stream stream);
+                         q4_dtype y_dtype, void* workspace, size_t workspace_bytes,
+                         q4_stream stream);
 
 /*
  * The same product for batches 1 <= B <= 128 (the skinny-GEMM regime of
@@ -146,7 +165,8 @@ Q4_API q4_status q4_gemv(const q4_weight* w, const void* x, q4_dtype x_dtype, in
  * requirements as q4_gemv.
  */
 Q4_API q4_status q4_gemm_skinny(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B,
-                         void* y, q4_dtype y_dtype, q4_stream stream);
+                                void* y, q4_dtype y_dtype, void* workspace,
+                                size_t workspace_bytes, q4_stream stream);
 
 /*
  * The unquantised bf16 product y = x W^T with fp32 accumulation, the

@@ -27,6 +27,7 @@ Q4_ERR_ALIGNMENT = 3
 Q4_ERR_UNSUPPORTED = 4
 Q4_ERR_CUDA = 5
 Q4_ERR_TIMEOUT = 6
+Q4_ERR_WORKSPACE = 7
 
 Q4_F16, Q4_BF16, Q4_F32 = 0, 1, 2
 _DT = {torch.float16: Q4_F16, torch.bfloat16: Q4_BF16, torch.float32: Q4_F32}
@@ -35,6 +36,7 @@ _DT = {torch.float16: Q4_F16, torch.bfloat16: Q4_BF16, torch.float32: Q4_F32}
 ABI_SYMBOLS = (
     "q4_quantize_pack", "q4_dequant", "q4_gemv", "q4_gemm_skinny", "bf16_gemv_ref_bw",
     "q4_sync_status", "q4_status_string", "q4_version", "q4_selftest_wait_timeout",
+    "q4_workspace_bytes",
 )
 
 
@@ -80,8 +82,10 @@ def load_library(path: str = LIB_PATH):
     W = ctypes.POINTER(_CWeight)
     lib.q4_quantize_pack.argtypes = [P, S, I64, I64, I32, I32, I32, P, P, P, P]
     lib.q4_dequant.argtypes = [W, P, S, P]
-    lib.q4_gemv.argtypes = [W, P, S, I64, P, S, P]
-    lib.q4_gemm_skinny.argtypes = [W, P, S, I64, P, S, P]
+    lib.q4_gemv.argtypes = [W, P, S, I64, P, S, P, ctypes.c_size_t, P]
+    lib.q4_gemm_skinny.argtypes = [W, P, S, I64, P, S, P, ctypes.c_size_t, P]
+    lib.q4_workspace_bytes.argtypes = [I64, I64, I64, I32]
+    lib.q4_workspace_bytes.restype = ctypes.c_size_t
     lib.bf16_gemv_ref_bw.argtypes = [P, I64, I64, P, I64, P, P]
     lib.q4_sync_status.argtypes = [P]
     lib.q4_selftest_wait_timeout.argtypes = [I64, P]
@@ -184,30 +188,51 @@ def q4_dequant(w: Q4Weight, out_dtype=torch.float32, W_hat: torch.Tensor | None 
     return W_hat
 
 
-def _product(fn_name: str, w: Q4Weight, x: torch.Tensor, y, y_dtype, stream):
+_workspaces: dict = {}
+
+
+def workspace_for(w: Q4Weight, B: int, device) -> torch.Tensor:
+    """A zero-filled device workspace large enough for q4_gemv / q4_gemm_skinny
+    on ``w`` with batch ``B``.  One buffer per device is kept and grown on
+    demand; every completed call leaves it zero-filled.  Calls that may
+    overlap on the GPU (different streams) must pass their own buffers."""
+    need = int(load_library().q4_workspace_bytes(w.out, w.in_features, B, w.group_size))
+    dev = torch.device(device)
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    buf = _workspaces.get(key)
+    if buf is None or buf.numel() < need:
+        buf = torch.zeros(max(need, 1 << 20), dtype=torch.uint8, device=dev)
+        _workspaces[key] = buf
+    return buf
+
+
+def _product(fn_name: str, w: Q4Weight, x: torch.Tensor, y, y_dtype, workspace, stream):
     lib = load_library()
     if x.dim() != 2:
         raise ValueError("x must be [B, in]")
     B = x.shape[0]
     if y is None:
         y = torch.empty(B, w.out, dtype=y_dtype or x.dtype, device=x.device)
+    if workspace is None:
+        workspace = workspace_for(w, B, x.device)
     cw = w.c_struct()
     st = getattr(lib, fn_name)(ctypes.byref(cw), _ptr(x), _DT[x.dtype], B, _ptr(y),
-                               _DT[y.dtype], _stream(stream))
+                               _DT[y.dtype], _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(stream))
     _check(st, fn_name)
     return y
 
 
 def q4_gemv(w: Q4Weight, x: torch.Tensor, y: torch.Tensor | None = None, y_dtype=None,
-            stream=None) -> torch.Tensor:
+            workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """y = x W_hat^T for B <= 8 (x [B, in] bf16/fp16; y [B, out] x.dtype or fp32)."""
-    return _product("q4_gemv", w, x, y, y_dtype, stream)
+    return _product("q4_gemv", w, x, y, y_dtype, workspace, stream)
 
 
 def q4_gemm_skinny(w: Q4Weight, x: torch.Tensor, y: torch.Tensor | None = None, y_dtype=None,
-                   stream=None) -> torch.Tensor:
+                   workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """y = x W_hat^T for B <= 128."""
-    return _product("q4_gemm_skinny", w, x, y, y_dtype, stream)
+    return _product("q4_gemm_skinny", w, x, y, y_dtype, workspace, stream)
 
 
 def bf16_gemv_ref_bw(W: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None,

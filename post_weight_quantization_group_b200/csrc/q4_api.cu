@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -13,6 +14,7 @@
 #include "q4.h"
 #include "q4_device.cuh"
 #include "q4_gemv.cuh"
+#include "q4_gemv_sk.cuh"
 #include "q4_quant.cuh"
 
 namespace {
@@ -81,9 +83,10 @@ EncodeTiledFn encode_fn() {
 }
 
 // 2-D row-major tensor [rows, cols] of `elem` bytes, box [box_rows, box_cols],
-// 128-byte swizzle, out-of-bounds elements read as zero.
+// out-of-bounds elements read as zero.
 bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem,
-                  uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols) {
+                  uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+                  CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {cols, rows};
@@ -91,7 +94,7 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, in
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -128,24 +131,41 @@ SplitPlan plan_split(int64_t out, int nchunks, int rt, int sms) {
     return {S, cps};
 }
 
+// Launch with an optional cluster shape and, for kernels written for it,
+// programmatic stream serialization (the kernel may start before the previous
+// kernel of the stream has finished; it waits with griddepcontrol.wait).
 template <typename... KArgs, typename... Args>
-q4_status launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                         int cluster_x, cudaStream_t stream, Args&&... args) {
+q4_status launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                    int cluster_x, bool pdl, cudaStream_t stream, Args&&... args) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    int n = 0;
     if (cluster_x > 1) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = cluster_x;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
     }
+    if (pdl) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    cfg.attrs = n ? attr : nullptr;
+    cfg.numAttrs = n;
     return launch_status(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
+}
+
+template <typename... KArgs, typename... Args>
+q4_status launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                         int cluster_x, cudaStream_t stream, Args&&... args) {
+    return launch_ex(kernel, grid, block, smem, cluster_x, false, stream,
+                     std::forward<Args>(args)...);
 }
 
 bool valid_dtype(int d) { return d == Q4_F16 || d == Q4_BF16 || d == Q4_F32; }
@@ -207,58 +227,120 @@ q4_status run_quantize(const void* W, int64_t out, int64_t in, int g, uint8_t* q
 }
 
 // ------------------------------------------------------------------ GEMV
-constexpr int kGemvMT = 2;
-constexpr int kGemvCW = 4;
-constexpr int kGemvStages = 4;
+// Tile shape of the small-batch kernels (compile-time tunables).
+#ifndef Q4_GEMV_MT
+#define Q4_GEMV_MT 2
+#endif
+#ifndef Q4_GEMV_CW
+#define Q4_GEMV_CW 4
+#endif
+#ifndef Q4_GEMV_STAGES
+#define Q4_GEMV_STAGES 4
+#endif
+constexpr int kGemvMT = Q4_GEMV_MT;
+constexpr int kGemvCW = Q4_GEMV_CW;
+constexpr int kGemvStages = Q4_GEMV_STAGES;
 constexpr int kGemvRT = kGemvCW * kGemvMT * 16;
 
-template <bool BF16, int GS, bool SYM>
-q4_status run_gemv(const q4_weight* w, const void* x, int64_t B, void* y, int ydt,
-                   cudaStream_t st) {
-    const int dev = current_device();
-    const int sms = sm_count(dev);
-    const int nchunks = static_cast<int>((w->in + kChunkCodes - 1) / kChunkCodes);
-    SplitPlan p = plan_split(w->out, nchunks, kGemvRT, sms);
-    GemvGeom geo = gemv_geom(kGemvRT, kGemvStages, p.cps, static_cast<int>(B), GS, SYM);
-    const int smax = max_smem_optin(dev);
-    while (geo.total > static_cast<size_t>(smax) && p.S < 16) {
-        p.S = p.S * 2 > 16 ? 16 : p.S * 2;
-        p.cps = (nchunks + p.S - 1) / p.S;
-        p.S = (nchunks + p.cps - 1) / p.cps;
-        geo = gemv_geom(kGemvRT, kGemvStages, p.cps, static_cast<int>(B), GS, SYM);
-        if (p.S == 16 || p.cps == 1) break;
-    }
-    if (geo.total > static_cast<size_t>(smax)) return Q4_ERR_UNSUPPORTED;
+// Small-batch stream-K kernel: CW consumer warps (16 rows each), 2 CTAs/SM.
+#ifndef Q4_SK_CW
+#define Q4_SK_CW 8
+#endif
+constexpr int kSkCW = Q4_SK_CW;
+constexpr int kSkRT = kSkCW * 16;
+constexpr int kSkCtasPerSm = 2;
+constexpr int kSkMinIters = 4;
 
-    CUtensorMap tmap;
-    if (!make_tmap_2d(&tmap, w->qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
-                      static_cast<uint64_t>(w->out), static_cast<uint64_t>(w->in / 2),
-                      kGemvRT, kChunkBytes))
+// Workspace layout, the same for every shape on a device so that one buffer
+// can serve calls of any shape: [partial slots of the largest grid]
+// [one counter per row tile].  Counters are reset by every call that uses
+// them; partial slots never overlap counters.
+struct SkPlan {
+    int64_t row_tiles, T, P;
+    int nchunks;
+    size_t ws_part_bytes, ws_bytes;
+};
+
+SkPlan sk_plan(int64_t out, int64_t in, int sms) {
+    SkPlan p{};
+    const int64_t pmax = static_cast<int64_t>(kSkCtasPerSm) * sms;
+    p.nchunks = static_cast<int>((in + kChunkCodes - 1) / kChunkCodes);
+    p.row_tiles = (out + kSkRT - 1) / kSkRT;
+    p.T = p.row_tiles * p.nchunks;
+    // at least kSkMinIters iterations per CTA: tiny problems use fewer SMs
+    // rather than paying a fixup for every chunk
+    p.P = std::min<int64_t>(std::max<int64_t>(1, p.T / kSkMinIters), pmax);
+    p.ws_part_bytes = static_cast<size_t>(2 * pmax) * kSkRT * 8 * 4;
+    p.ws_bytes = p.ws_part_bytes + align_up(static_cast<size_t>(p.row_tiles) * 4, 256);
+    return p;
+}
+
+template <bool BF16, int GS, bool SYM>
+q4_status run_gemv(const q4_weight* w, const void* x, int64_t B, void* y, int ydt, void* ws,
+                   size_t ws_bytes, cudaStream_t st) {
+    const int dev = current_device();
+    const SkPlan p = sk_plan(w->out, w->in, sm_count(dev));
+    if (!ws || ws_bytes < p.ws_bytes) return Q4_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return Q4_ERR_ALIGNMENT;
+    // deepest ring that still lets two CTAs share an SM
+    const int per_sm = 228 * 1024;
+    int stages = kSkMaxStages;
+    SkGeom geo = sk_geom(kSkRT, stages, static_cast<int>(B), SYM);
+    while (stages > 2 && kSkCtasPerSm * (geo.total + 1024) > static_cast<size_t>(per_sm)) {
+        --stages;
+        geo = sk_geom(kSkRT, stages, static_cast<int>(B), SYM);
+    }
+    const int64_t G = w->in / GS;
+    // scale / zero windows by TMA when their rows are 16-byte aligned
+    const bool meta_tma = (G % 8) == 0 && aligned(w->scales, 16) && (SYM || aligned(w->zeros, 16));
+    CUtensorMap tmap_w, tmap_x, tmap_s, tmap_z;
+    std::memset(&tmap_s, 0, sizeof(tmap_s));
+    std::memset(&tmap_z, 0, sizeof(tmap_z));
+    if (!make_tmap_2d(&tmap_w, w->qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                      static_cast<uint64_t>(w->out), static_cast<uint64_t>(w->in / 2), kSkRT,
+                      kChunkBytes))
         return Q4_ERR_CUDA;
-    auto kernel = q4_gemv_kernel<BF16, GS, SYM, kGemvMT, kGemvCW, kGemvStages>;
-    if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), p.S > 8)) return Q4_ERR_CUDA;
+    if (!make_tmap_2d(&tmap_x, x,
+                      BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                      static_cast<uint64_t>(B), static_cast<uint64_t>(w->in),
+                      static_cast<uint32_t>(B), kChunkCodes, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return Q4_ERR_CUDA;
+    if (meta_tma) {
+        if (!make_tmap_2d(&tmap_s, w->scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                          static_cast<uint64_t>(w->out), static_cast<uint64_t>(G), kSkRT, 8,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+            return Q4_ERR_CUDA;
+        if (!SYM && !make_tmap_2d(&tmap_z, w->zeros, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                                  static_cast<uint64_t>(w->out), static_cast<uint64_t>(G), kSkRT,
+                                  8, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return Q4_ERR_CUDA;
+    }
+    auto kernel = q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW>;
+    if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), false)) return Q4_ERR_CUDA;
     unsigned* status = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
         return Q4_ERR_CUDA;
-    const dim3 grid(p.S, static_cast<unsigned>((w->out + kGemvRT - 1) / kGemvRT));
-    return launch_cluster(kernel, grid, dim3((kGemvCW + 1) * 32), geo.total, p.S, st, tmap,
-                          reinterpret_cast<const __half*>(w->scales),
-                          reinterpret_cast<const __half*>(w->zeros),
-                          reinterpret_cast<const uint16_t*>(x), static_cast<int>(B), w->out,
-                          w->in, p.cps, nchunks, y, ydt, status);
+    float* ws_part = reinterpret_cast<float*>(ws);
+    unsigned* ws_count = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(ws) + p.ws_part_bytes);
+    return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3((kSkCW + 2) * 32),
+                          geo.total, 1, true, st, tmap_w, tmap_x, tmap_s, tmap_z, meta_tma ? 1 : 0,
+                          reinterpret_cast<const uint16_t*>(w->scales),
+                          reinterpret_cast<const uint16_t*>(w->zeros), stages,
+                          static_cast<int>(B), w->out, w->in, p.nchunks, p.T, y, ydt, ws_part,
+                          ws_count, status);
 }
 
 template <bool BF16>
-q4_status dispatch_gemv(const q4_weight* w, const void* x, int64_t B, void* y, int ydt,
-                        cudaStream_t st) {
+q4_status dispatch_gemv(const q4_weight* w, const void* x, int64_t B, void* y, int ydt, void* ws,
+                        size_t wsb, cudaStream_t st) {
     const bool sym = w->symmetric != 0;
     switch (w->group_size) {
-        case 32: return sym ? run_gemv<BF16, 32, true>(w, x, B, y, ydt, st)
-                            : run_gemv<BF16, 32, false>(w, x, B, y, ydt, st);
-        case 64: return sym ? run_gemv<BF16, 64, true>(w, x, B, y, ydt, st)
-                            : run_gemv<BF16, 64, false>(w, x, B, y, ydt, st);
-        case 128: return sym ? run_gemv<BF16, 128, true>(w, x, B, y, ydt, st)
-                             : run_gemv<BF16, 128, false>(w, x, B, y, ydt, st);
+        case 32: return sym ? run_gemv<BF16, 32, true>(w, x, B, y, ydt, ws, wsb, st)
+                            : run_gemv<BF16, 32, false>(w, x, B, y, ydt, ws, wsb, st);
+        case 64: return sym ? run_gemv<BF16, 64, true>(w, x, B, y, ydt, ws, wsb, st)
+                            : run_gemv<BF16, 64, false>(w, x, B, y, ydt, ws, wsb, st);
+        case 128: return sym ? run_gemv<BF16, 128, true>(w, x, B, y, ydt, ws, wsb, st)
+                             : run_gemv<BF16, 128, false>(w, x, B, y, ydt, ws, wsb, st);
         default: return Q4_ERR_UNSUPPORTED;
     }
 }
@@ -297,6 +379,7 @@ const char* q4_status_string(q4_status s) {
         case Q4_ERR_UNSUPPORTED: return "Q4_ERR_UNSUPPORTED";
         case Q4_ERR_CUDA: return "Q4_ERR_CUDA";
         case Q4_ERR_TIMEOUT: return "Q4_ERR_TIMEOUT";
+        case Q4_ERR_WORKSPACE: return "Q4_ERR_WORKSPACE";
     }
     return "Q4_ERR_UNKNOWN";
 }
@@ -371,22 +454,31 @@ q4_status q4_dequant(const q4_weight* w, void* W_hat, q4_dtype out_dtype, q4_str
     return launch_status(cudaSuccess);
 }
 
+size_t q4_workspace_bytes(int64_t out, int64_t in, int64_t B, int32_t group_size) {
+    if (out < 0 || in <= 0 || B < 1 || B > 128 || group_size <= 0) return 0;
+    if (out == 0) return 0;
+    return sk_plan(out, in, sm_count(current_device())).ws_bytes;
+}
+
 q4_status q4_gemv(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B, void* y,
-                  q4_dtype y_dtype, q4_stream stream) {
+                  q4_dtype y_dtype, void* workspace, size_t workspace_bytes, q4_stream stream) {
     q4_status s = validate_product(w, x, x_dtype, B, y, y_dtype, 8);
     if (s != Q4_OK) return s;
     if (w->out == 0) return Q4_OK;
+    if (!workspace) return Q4_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int ydt = y_dtype == Q4_F32 ? 2 : (y_dtype == Q4_BF16 ? 1 : 0);
-    return x_dtype == Q4_BF16 ? dispatch_gemv<true>(w, x, B, y, ydt, st)
-                              : dispatch_gemv<false>(w, x, B, y, ydt, st);
+    return x_dtype == Q4_BF16
+               ? dispatch_gemv<true>(w, x, B, y, ydt, workspace, workspace_bytes, st)
+               : dispatch_gemv<false>(w, x, B, y, ydt, workspace, workspace_bytes, st);
 }
 
 q4_status q4_gemm_skinny(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B,
-                         void* y, q4_dtype y_dtype, q4_stream stream) {
+                         void* y, q4_dtype y_dtype, void* workspace, size_t workspace_bytes,
+                         q4_stream stream) {
     q4_status s = validate_product(w, x, x_dtype, B, y, y_dtype, 128);
     if (s != Q4_OK) return s;
-    if (B <= 8) return q4_gemv(w, x, x_dtype, B, y, y_dtype, stream);
+    if (B <= 8) return q4_gemv(w, x, x_dtype, B, y, y_dtype, workspace, workspace_bytes, stream);
     return Q4_ERR_UNSUPPORTED;
 }
 

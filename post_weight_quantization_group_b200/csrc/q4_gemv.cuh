@@ -11,15 +11,19 @@
 //  * one producer warp streams [RT rows x 128 B] tiles of the packed weights
 //    into a ring of shared-memory stages with TMA (128-byte swizzle), paced by
 //    full / empty mbarriers;
-//  * consumer warps unpack each 32-bit word (8 codes) into exact 16-bit
-//    integers with LOP3 magic-number conversion (code | 0x4300 is the bf16
-//    value 128 + code), subtract the offset (8 for two's-complement symmetric
-//    codes, z for asymmetric ones), and feed them as the A operand of
-//    m16n8k16 tensor-core MMAs whose B operand is the activation batch (n = 8
-//    columns, B of them live).  Products of small integers with 16-bit
-//    activations are exact, the MMA accumulates them in fp32 over one group,
-//    and the group's partial sum is multiplied by its fp32 scale and added to
-//    the running fp32 accumulator;
+//  * consumer warps turn each 32-bit word (8 codes) into exact 16-bit
+//    integers with one LOP3 per code pair: code | 0x4300 is the bf16 value
+//    128 + code (0x6400: fp16 1024 + code; symmetric codes are XORed with 8
+//    in the same LOP3 to make them 0..15).  These raw values are the A
+//    operand of m16n8k16 tensor-core MMAs whose B operand is the activation
+//    batch (n = 8 columns, B of them live).  The products are exact and the
+//    MMA accumulates one group in fp32; the constant offset is removed per
+//    group as  sum (c + q') x = c * sum x + sum q' x,  with c = 136 (bf16,
+//    symmetric), 128 + z (bf16, asymmetric) or 1024 + 8 / 1024 + z (fp16) and
+//    sum x of the group precomputed once per CTA.  The accumulator restarts
+//    every group, so the cancellation costs about 6 (bf16) to 9 (fp16) of
+//    fp32's 24 bits on one group's partial; the partial is then multiplied
+//    by the group's fp32 scale and added to the running fp32 accumulator;
 //  * the K dimension is split over the CTAs of a thread-block cluster; each
 //    CTA leaves its [RT x B] fp32 partial in shared memory and the cluster
 //    reduces them through distributed shared memory, in rank order, so the
@@ -48,14 +52,17 @@ struct GemvGeom {
     int cps;          // chunks per split
     int b;            // batch
     int gpc;          // groups per chunk
+    int glp;          // groups per CTA, padded to a multiple of 8 (16 bytes of fp16)
     bool sym;
     // byte offsets in dynamic shared memory
-    size_t off_x, off_s, off_z, off_bar, total;
+    size_t off_x, off_s, off_z, off_sx, off_bar, total;
 };
 
 // Chunk = 256 codes of a row = 128 bytes.
 constexpr int kChunkCodes = 256;
 constexpr int kChunkBytes = 128;
+
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 __host__ __device__ inline GemvGeom gemv_geom(int rt, int stages, int cps, int b, int gs,
                                               bool sym) {
@@ -65,17 +72,20 @@ __host__ __device__ inline GemvGeom gemv_geom(int rt, int stages, int cps, int b
     g.cps = cps;
     g.b = b;
     g.gpc = kChunkCodes / gs;
+    g.glp = static_cast<int>(align_up(static_cast<size_t>(cps) * g.gpc, 8));
     g.sym = sym;
     size_t off = static_cast<size_t>(stages) * rt * kChunkBytes;  // stages, 1024-aligned
     g.off_x = off;
     off += static_cast<size_t>(b) * cps * 512;                     // permuted x
-    g.off_s = off;
-    off += static_cast<size_t>(cps) * g.gpc * rt * 2;              // scales (fp16 pairs)
-    g.off_z = off;
-    if (!sym) off += static_cast<size_t>(cps) * g.gpc * rt * 2;    // zeros
-    off = (off + 15) & ~static_cast<size_t>(15);
+    off = align_up(off, 1024);
+    g.off_s = off;                                                 // scales [rt][glp] fp16
+    off = align_up(off + static_cast<size_t>(rt) * g.glp * 2, 1024);
+    g.off_z = off;                                                 // zeros  [rt][glp] fp16
+    if (!sym) off = align_up(off + static_cast<size_t>(rt) * g.glp * 2, 1024);
+    g.off_sx = off;                                                // group sums of x [glp][8] fp32
+    off += static_cast<size_t>(g.glp) * 8 * 4;
     g.off_bar = off;
-    off += static_cast<size_t>(2 * stages) * 8;
+    off += static_cast<size_t>(2 * stages + 1) * 8;
     g.total = off + 1024;  // slack to align the base to 1024 bytes
     return g;
 }
@@ -132,10 +142,12 @@ __device__ __forceinline__ void cluster_reduce_store(const float* red, int rt, i
 // grid = (S splits of K, ceil(out / RT)); cluster = (S, 1, 1) when S > 1.
 template <bool BF16, int GS, bool SYM, int MT, int CW, int STAGES>
 __global__ void __launch_bounds__((CW + 1) * 32)
-    q4_gemv_kernel(const __grid_constant__ CUtensorMap tmap_w, const __half* __restrict__ scales,
-                   const __half* __restrict__ zeros, const uint16_t* __restrict__ x, int B,
-                   int64_t out, int64_t in, int cps, int nchunks, void* __restrict__ y, int ydt,
-                   unsigned* __restrict__ status) {
+    q4_gemv_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                   const __grid_constant__ CUtensorMap tmap_s,
+                   const __grid_constant__ CUtensorMap tmap_z, int meta_tma,
+                   const __half* __restrict__ scales, const __half* __restrict__ zeros,
+                   const uint16_t* __restrict__ x, int B, int64_t out, int64_t in, int cps,
+                   int nchunks, void* __restrict__ y, int ydt, unsigned* __restrict__ status) {
     constexpr int RT = CW * MT * 16;
     constexpr int GPC = kChunkCodes / GS;  // groups per chunk
     constexpr int WPG = GS / 32;           // 32-bit words per thread per row per group
@@ -147,10 +159,13 @@ __global__ void __launch_bounds__((CW + 1) * 32)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const GemvGeom geo = gemv_geom(RT, STAGES, cps, B, GS, SYM);
     uint8_t* xs = smem + geo.off_x;
-    uint32_t* ss = reinterpret_cast<uint32_t*>(smem + geo.off_s);
-    uint32_t* zs = reinterpret_cast<uint32_t*>(smem + geo.off_z);
+    uint16_t* ss16 = reinterpret_cast<uint16_t*>(smem + geo.off_s);
+    uint16_t* zs16 = reinterpret_cast<uint16_t*>(smem + geo.off_z);
+    float* sxs = reinterpret_cast<float*>(smem + geo.off_sx);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + geo.off_bar);
     uint64_t* empty = full + STAGES;
+    uint64_t* meta = empty + STAGES;  // scales / zeros tile landed
+    const int GLP = geo.glp;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -165,6 +180,7 @@ __global__ void __launch_bounds__((CW + 1) * 32)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], CW);
         }
+        mbar_init(meta, 1);
         fence_mbarrier_init_cluster();
     }
     __syncthreads();
@@ -179,6 +195,13 @@ __global__ void __launch_bounds__((CW + 1) * 32)
         // ------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tmap_w);
+            if (meta_tma && nch > 0) {
+                // the CTA's [RT x GLP] scale (and zero) tiles, group index c_begin*GPC
+                mbar_arrive_expect_tx(meta, RT * GLP * 2 * (SYM ? 1 : 2));
+                tma_load_2d(ss16, &tmap_s, c_begin * GPC, static_cast<int32_t>(row0), meta);
+                if constexpr (!SYM)
+                    tma_load_2d(zs16, &tmap_z, c_begin * GPC, static_cast<int32_t>(row0), meta);
+            }
             bool ok = true;
             for (int c = 0; c < nch && ok; ++c) {
                 const int s = c % STAGES;
@@ -190,6 +213,7 @@ __global__ void __launch_bounds__((CW + 1) * 32)
                 tma_load_2d(smem + static_cast<size_t>(s) * RT * kChunkBytes, &tmap_w,
                             (c_begin + c) * kChunkBytes, static_cast<int32_t>(row0), &full[s]);
             }
+            if (meta_tma && nch > 0) mbar_wait_bounded(meta, 0, status, kWaitLimitNs);
             // drain: the last phase of every stage that was filled must have
             // landed before shared memory is reused or released
             for (int s = 0; s < STAGES && s < nch; ++s) {
@@ -202,48 +226,106 @@ __global__ void __launch_bounds__((CW + 1) * 32)
         // ------------------------------------------------------ consumers
         const int ctid = threadIdx.x;  // 0 .. CW*32-1
         // permuted activations: block p of chunk c for batch n goes to word
-        // slot w = G*WPG + i of thread t, where p = G*(GS/8) + t*WPG + i
+        // slot w = G*WPG + i of thread t, where p = G*(GS/8) + t*WPG + i.
+        // All loads of a batch are issued before any store.
         const int kbase = c_begin * kChunkCodes;
-        for (int idx = ctid; idx < B * nch * 32; idx += CW * 32) {
-            const int p = idx & 31;
-            const int c = (idx >> 5) % nch;
-            const int n = (idx >> 5) / nch;
-            const int64_t k = static_cast<int64_t>(kbase) + c * kChunkCodes + p * 8;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (k < in) v = __ldg(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(n) * in + k));
-            uint4 o;
-            o.x = prmt(v.x, v.z, 0x5410);  // (x0, x4)
-            o.y = prmt(v.x, v.z, 0x7632);  // (x1, x5)
-            o.z = prmt(v.y, v.w, 0x5410);  // (x2, x6)
-            o.w = prmt(v.y, v.w, 0x7632);  // (x3, x7)
-            const int gq = p / (GS / 8);
-            const int rem = p % (GS / 8);
-            const int t = rem / WPG;
-            const int i = rem % WPG;
-            const int w = gq * WPG + i;
-            *reinterpret_cast<uint4*>(xs + ((static_cast<size_t>(c) * 8 + w) * B + n) * 64 + 16 * t) = o;
-        }
-        // scales / zeros as (row r0, row r0 + 8) pairs per (group, m-tile, lane group)
-        const int GL = nch * GPC;
-        const int64_t gbase = static_cast<int64_t>(c_begin) * GPC;
-        uint16_t* ss16 = reinterpret_cast<uint16_t*>(ss);
-        uint16_t* zs16 = reinterpret_cast<uint16_t*>(zs);
-        for (int idx = ctid; idx < RT * GL; idx += CW * 32) {
-            const int gl = idx % GL;
-            const int r = idx / GL;
-            const int64_t grow = row0 + r;
-            const int64_t gg = gbase + gl;
-            uint16_t sv = 0, zv = 0;
-            if (grow < out && gg < G) {
-                sv = __half_as_ushort(scales[grow * G + gg]);
-                if constexpr (!SYM) zv = __half_as_ushort(zeros[grow * G + gg]);
+        const int nitems = B * nch * 32;
+        constexpr int XU = 4;
+        for (int base = ctid; base < nitems; base += XU * CW * 32) {
+            uint4 v[XU];
+#pragma unroll
+            for (int u = 0; u < XU; ++u) {
+                const int idx = base + u * CW * 32;
+                v[u] = make_uint4(0, 0, 0, 0);
+                if (idx < nitems) {
+                    const int p = idx & 31;
+                    const int c = (idx >> 5) % nch;
+                    const int n = (idx >> 5) / nch;
+                    const int64_t k = static_cast<int64_t>(kbase) + c * kChunkCodes + p * 8;
+                    if (k < in)
+                        v[u] = __ldg(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(n) * in + k));
+                }
             }
-            const int rr = r & 15;
-            const int slot = (((gl * (RT / 16) + (r >> 4)) * 8 + rho(rr & 7)) << 1) | (rr >> 3);
-            ss16[slot] = sv;
-            if constexpr (!SYM) zs16[slot] = zv;
+#pragma unroll
+            for (int u = 0; u < XU; ++u) {
+                const int idx = base + u * CW * 32;
+                if (idx < nitems) {
+                    const int p = idx & 31;
+                    const int c = (idx >> 5) % nch;
+                    const int n = (idx >> 5) / nch;
+                    uint4 o;
+                    o.x = prmt(v[u].x, v[u].z, 0x5410);  // (x0, x4)
+                    o.y = prmt(v[u].x, v[u].z, 0x7632);  // (x1, x5)
+                    o.z = prmt(v[u].y, v[u].w, 0x5410);  // (x2, x6)
+                    o.w = prmt(v[u].y, v[u].w, 0x7632);  // (x3, x7)
+                    const int gq = p / (GS / 8);
+                    const int rem = p % (GS / 8);
+                    const int t = rem / WPG;
+                    const int i = rem % WPG;
+                    const int w = gq * WPG + i;
+                    *reinterpret_cast<uint4*>(xs + ((static_cast<size_t>(c) * 8 + w) * B + n) * 64 + 16 * t) = o;
+                }
+            }
+        }
+        if (!meta_tma) {
+            // scales / zeros whose rows are not 16-byte aligned: plain loads into
+            // the same [RT][GLP] layout the tensor-map copy produces
+            const int GL = nch * GPC;
+            const int64_t gbase = static_cast<int64_t>(c_begin) * GPC;
+            for (int idx = ctid; idx < RT * GLP; idx += CW * 32) {
+                const int gl = idx % GLP;
+                const int r = idx / GLP;
+                const int64_t grow = row0 + r;
+                const int64_t gg = gbase + gl;
+                uint16_t sv = 0, zv = 0;
+                if (gl < GL && grow < out && gg < G) {
+                    sv = __half_as_ushort(scales[grow * G + gg]);
+                    if constexpr (!SYM) zv = __half_as_ushort(zeros[grow * G + gg]);
+                }
+                ss16[idx] = sv;
+                if constexpr (!SYM) zs16[idx] = zv;
+            }
         }
         named_bar_sync(1, CW * 32);
+        // per (group, batch) sums of the activations, in a fixed order
+        {
+            const int GL = nch * GPC;
+            for (int idx = ctid; idx < GLP * 8; idx += CW * 32) {
+                const int gl = idx >> 3;
+                const int n = idx & 7;
+                float sum = 0.f;
+                if (n < B && gl < GL) {
+                    const int c = gl / GPC;
+                    const int gq = gl % GPC;
+#pragma unroll
+                    for (int i = 0; i < WPG; ++i) {
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const uint4 v = *reinterpret_cast<const uint4*>(
+                                xs + ((static_cast<size_t>(c) * 8 + gq * WPG + i) * B + n) * 64 + 16 * t);
+                            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                float lo, hi;
+                                if constexpr (BF16) {
+                                    lo = __uint_as_float(wv[e] << 16);
+                                    hi = __uint_as_float(wv[e] & 0xFFFF0000u);
+                                } else {
+                                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[e]));
+                                    lo = f.x;
+                                    hi = f.y;
+                                }
+                                sum += lo;
+                                sum += hi;
+                            }
+                        }
+                    }
+                }
+                sxs[idx] = sum;
+            }
+        }
+        named_bar_sync(1, CW * 32);
+        if (meta_tma && nch > 0) mbar_wait_bounded(meta, 0, status, kWaitLimitNs);
 
         const int gid = lane >> 2;
         const int t = lane & 3;
@@ -273,6 +355,8 @@ __global__ void __launch_bounds__((CW + 1) * 32)
                         xf[i][0] = xf[i][1] = xf[i][2] = xf[i][3] = 0u;
                     }
                 }
+                // group sums for this lane's accumulator columns n = 2t, 2t+1
+                const float2 sx = *reinterpret_cast<const float2*>(sxs + (c * GPC + gq) * 8 + 2 * t);
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
                     const int mtile = warp * MT + mt;
@@ -299,44 +383,41 @@ __global__ void __launch_bounds__((CW + 1) * 32)
                         w0[0] = *reinterpret_cast<const uint32_t*>(p0);
                         w1[0] = *reinterpret_cast<const uint32_t*>(p1);
                     }
-                    const int sidx = ((c * GPC + gq) * (RT / 16) + mtile) * 8 + gid;
-                    const uint32_t sp = ss[sidx];
-                    const float2 sc = __half22float2(*reinterpret_cast<const __half2*>(&sp));
-                    uint32_t off0, off1;
+                    const int gl = c * GPC + gq;
+                    const float2 sc = make_float2(
+                        __half2float(__ushort_as_half(ss16[R0 * GLP + gl])),
+                        __half2float(__ushort_as_half(ss16[(R0 + 8) * GLP + gl])));
+                    // offset of the raw values: base + 8 (symmetric) or base + z
+                    float cst0, cst1;
                     if constexpr (SYM) {
-                        // (base + code + 8) - (base + 8) = code
-                        const uint16_t ob = small_int_bits<BF16>(Magic<BF16>::base + 8.0f);
-                        off0 = off1 = (static_cast<uint32_t>(ob) << 16) | ob;
+                        cst0 = cst1 = Magic<BF16>::base + 8.0f;
                     } else {
-                        const uint32_t zp = zs[sidx];
-                        const float2 zz = __half22float2(*reinterpret_cast<const __half2*>(&zp));
-                        const uint16_t o0 = small_int_bits<BF16>(Magic<BF16>::base + zz.x);
-                        const uint16_t o1 = small_int_bits<BF16>(Magic<BF16>::base + zz.y);
-                        off0 = (static_cast<uint32_t>(o0) << 16) | o0;
-                        off1 = (static_cast<uint32_t>(o1) << 16) | o1;
+                        cst0 = Magic<BF16>::base + __half2float(__ushort_as_half(zs16[R0 * GLP + gl]));
+                        cst1 = Magic<BF16>::base + __half2float(__ushort_as_half(zs16[(R0 + 8) * GLP + gl]));
                     }
-                    float part[4] = {0.f, 0.f, 0.f, 0.f};
+                    // two independent MMA accumulation chains per group
+                    float pa[4] = {0.f, 0.f, 0.f, 0.f};
+                    float pb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int i = 0; i < WPG; ++i) {
                         const uint32_t a = w0[i], b = w1[i];
                         // nibbles (0,4), (1,5), (2,6), (3,7) of each word
-                        const uint32_t lo0 = sub2<BF16>(lop3_and_xor(a, 0x000F000Fu, kMagic), off0);
-                        const uint32_t hi0 = sub2<BF16>(lop3_and_xor(a >> 4, 0x000F000Fu, kMagic), off0);
-                        const uint32_t lo20 = sub2<BF16>(lop3_and_xor(a >> 8, 0x000F000Fu, kMagic), off0);
-                        const uint32_t hi20 = sub2<BF16>(lop3_and_xor(a >> 12, 0x000F000Fu, kMagic), off0);
-                        const uint32_t lo1 = sub2<BF16>(lop3_and_xor(b, 0x000F000Fu, kMagic), off1);
-                        const uint32_t hi1 = sub2<BF16>(lop3_and_xor(b >> 4, 0x000F000Fu, kMagic), off1);
-                        const uint32_t lo21 = sub2<BF16>(lop3_and_xor(b >> 8, 0x000F000Fu, kMagic), off1);
-                        const uint32_t hi21 = sub2<BF16>(lop3_and_xor(b >> 12, 0x000F000Fu, kMagic), off1);
-                        const uint32_t A0[4] = {lo0, lo1, hi0, hi1};
-                        const uint32_t A1[4] = {lo20, lo21, hi20, hi21};
-                        mma_16816<BF16>(part, A0, xf[i][0], xf[i][1]);
-                        mma_16816<BF16>(part, A1, xf[i][2], xf[i][3]);
+                        const uint32_t A0[4] = {lop3_and_xor(a, 0x000F000Fu, kMagic),
+                                                lop3_and_xor(b, 0x000F000Fu, kMagic),
+                                                lop3_and_xor(a >> 4, 0x000F000Fu, kMagic),
+                                                lop3_and_xor(b >> 4, 0x000F000Fu, kMagic)};
+                        const uint32_t A1[4] = {lop3_and_xor(a >> 8, 0x000F000Fu, kMagic),
+                                                lop3_and_xor(b >> 8, 0x000F000Fu, kMagic),
+                                                lop3_and_xor(a >> 12, 0x000F000Fu, kMagic),
+                                                lop3_and_xor(b >> 12, 0x000F000Fu, kMagic)};
+                        mma_16816<BF16>(pa, A0, xf[i][0], xf[i][1]);
+                        mma_16816<BF16>(pb, A1, xf[i][2], xf[i][3]);
                     }
-                    acc[mt][0] = fmaf(sc.x, part[0], acc[mt][0]);
-                    acc[mt][1] = fmaf(sc.x, part[1], acc[mt][1]);
-                    acc[mt][2] = fmaf(sc.y, part[2], acc[mt][2]);
-                    acc[mt][3] = fmaf(sc.y, part[3], acc[mt][3]);
+                    // sum (c + q') x  ->  sum q' x  (q' = q - z), then scale
+                    acc[mt][0] = fmaf(sc.x, fmaf(-cst0, sx.x, pa[0] + pb[0]), acc[mt][0]);
+                    acc[mt][1] = fmaf(sc.x, fmaf(-cst0, sx.y, pa[1] + pb[1]), acc[mt][1]);
+                    acc[mt][2] = fmaf(sc.y, fmaf(-cst1, sx.x, pa[2] + pb[2]), acc[mt][2]);
+                    acc[mt][3] = fmaf(sc.y, fmaf(-cst1, sx.y, pa[3] + pb[3]), acc[mt][3]);
                 }
             }
             __syncwarp();

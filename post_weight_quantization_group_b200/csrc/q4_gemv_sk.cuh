@@ -1,0 +1,477 @@
+// q4_gemv_sk.cuh -- persistent stream-K W4A16 decode product for B <= 8.
+//
+//   y[b, r] = sum_j s[r, j] * sum_{k in group j} (q[r, k] - z[r, j]) * x[b, k]
+//
+// Work decomposition.  The product is T = row_tiles x chunks iterations (a
+// row tile is RT = 16 * CW rows, a chunk 256 codes of K).  A persistent grid
+// of P CTAs (two per SM) gives CTA p the contiguous range
+// [T p / P, T (p+1) / P) in tile-major order, so every CTA streams the same
+// number of bytes whatever the shape.  A range covers whole row tiles and at
+// most two partial ones.  A partial tile's fp32 partial goes to a workspace
+// slot; the CTA that arrives last on the tile's counter adds all partials of
+// the tile in CTA order -- the result does not depend on timing -- writes y
+// and resets the counter, so the counters are zero again for the next call.
+// No CTA ever waits for another.
+//
+// Launch overlap: the kernel lets the next kernel of the stream launch as
+// soon as it has started (programmatic dependent launch), and itself issues
+// the loads of its first stages of weights and scales -- which no preceding
+// kernel of this library writes -- before waiting for the preceding kernel;
+// activations, outputs and the workspace are touched only after that wait.
+//
+// Warp roles inside a CTA:
+//  * CW consumer warps, one 16-row MMA tile each;
+//  * a producer warp: one thread issues, per iteration, TMA loads of the
+//    weight tile [RT rows x 128 B] (128-byte swizzle), the activation chunk
+//    [B rows x 256 values] and the aligned window of 8 groups of scales
+//    (and zero points) [RT rows x 8] that holds the chunk's groups, into a
+//    ring of `stages` shared-memory stages;
+//  * a helper warp: per stage it rewrites the activation chunk in MMA
+//    fragment order and sums it per group, shared memory to shared memory,
+//    so the consumer threads do nothing but unpack, multiply and rescale.
+//    (Scale rows that are not 16-byte aligned cannot be copied by TMA; the
+//    helper then loads the chunk's scales itself.)
+//
+// Arithmetic (arganzheng.life post-training-quantization-gptq-awq-and-rotation,
+// section 二.3: codes unpacked on chip and multiplied on 16-bit tensor cores;
+// section 二.2: per-group scales applied inside the K accumulation): one LOP3
+// turns a code pair into the bf16 (fp16) values 128 + q' (1024 + q'), q' =
+// q + 8 for two's-complement symmetric codes and q' = q for asymmetric ones;
+// m16n8k16 MMAs multiply them exactly with the activations and accumulate one
+// group in fp32; the offset is removed per group as
+//   sum (c + q') x - c * sum x,   c = 136 | 128 + z (bf16), 1032 | 1024 + z (fp16),
+// and the group partial is multiplied by its fp32 scale.  The accumulator
+// restarts every group, so the cancellation costs 6 (bf16) to 9 (fp16) of
+// fp32's 24 bits of one group's partial.  Codes meet activations out of
+// natural order inside a group: each thread takes 8 consecutive codes per
+// 32-bit word and pairs nibbles (0,4), (1,5), (2,6), (3,7), and the helper
+// stores the activations in the matching order.
+#pragma once
+
+#include "q4_device.cuh"
+#include "q4_gemv.cuh"
+
+namespace q4dev {
+
+constexpr int kSkMaxStages = 4;
+
+struct SkGeom {
+    size_t off_x, off_xp, off_sx, off_sc, off_zc, stage_bytes, off_bar, total;
+};
+
+// Per stage: weights [rt x 128 B] | activations as loaded [b x 512 B] |
+// activations in fragment order [8 slots x 8 batch x 4 threads x 16 B] |
+// group sums [8 groups x 8 batch] fp32 | scale window [rt x 8] fp16 |
+// zero-point window [rt x 8] fp16 (asymmetric only).
+__host__ __device__ inline SkGeom sk_geom(int rt, int stages, int b, bool sym) {
+    SkGeom g{};
+    g.off_x = static_cast<size_t>(rt) * kChunkBytes;
+    g.off_xp = g.off_x + align_up(static_cast<size_t>(b) * 512, 128);
+    g.off_sx = g.off_xp + 8 * 8 * 64;
+    g.off_sc = g.off_sx + 8 * 8 * 4;
+    g.off_zc = g.off_sc + static_cast<size_t>(rt) * 16;
+    const size_t end = g.off_zc + (sym ? 0 : static_cast<size_t>(rt) * 16);
+    g.stage_bytes = align_up(end, 1024);
+    g.off_bar = g.stage_bytes * stages;
+    g.total = g.off_bar + static_cast<size_t>(3 * kSkMaxStages) * 8 + 64 + 1024;
+    return g;
+}
+
+// CTA that owns iteration i of T split over P CTAs: it_beg(q) = T q / P.
+__device__ __forceinline__ int64_t sk_owner(int64_t i, int64_t T, int64_t P) {
+    return ((i + 1) * P - 1) / T;
+}
+
+__device__ __forceinline__ uint32_t pair_lo(uint32_t a, uint32_t b) { return prmt(a, b, 0x5410); }
+__device__ __forceinline__ uint32_t pair_hi(uint32_t a, uint32_t b) { return prmt(a, b, 0x7632); }
+
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "l"(p), "r"(v)
+                 : "memory");
+    return old;
+}
+
+template <bool BF16, int GS, bool SYM, int CW>
+__global__ void __launch_bounds__((CW + 2) * 32, 2)
+    q4_gemv_sk_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                      const __grid_constant__ CUtensorMap tmap_x,
+                      const __grid_constant__ CUtensorMap tmap_s,
+                      const __grid_constant__ CUtensorMap tmap_z, int meta_tma,
+                      const uint16_t* __restrict__ scales, const uint16_t* __restrict__ zeros,
+                      int stages, int B, int64_t out, int64_t in, int nchunks, int64_t T,
+                      void* __restrict__ y, int ydt, float* __restrict__ ws_part,
+                      unsigned* __restrict__ ws_count, unsigned* __restrict__ status) {
+    constexpr int RT = CW * 16;
+    constexpr int GPC = kChunkCodes / GS;  // groups per chunk
+    constexpr int WPG = GS / 32;           // 32-bit words per thread per row per group
+    constexpr uint32_t kMagic = Magic<BF16>::base2 ^ (SYM ? 0x00080008u : 0u);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const SkGeom geo = sk_geom(RT, stages, B, SYM);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + geo.off_bar);
+    uint64_t* sxful = full + kSkMaxStages;
+    uint64_t* empty = sxful + kSkMaxStages;
+    unsigned* last_flag = reinterpret_cast<unsigned*>(empty + kSkMaxStages);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t P = gridDim.x;
+    const int64_t p = blockIdx.x;
+    const int64_t it_beg = (T * p) / P;
+    const int64_t it_end = (T * (p + 1)) / P;
+    const int nit = static_cast<int>(it_end - it_beg);
+    const int64_t G = in / GS;
+    const int tile0 = static_cast<int>(it_beg / nchunks);
+    const int chunk0 = static_cast<int>(it_beg - static_cast<int64_t>(tile0) * nchunks);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&sxful[s], 1);
+            mbar_init(&empty[s], CW);
+        }
+        fence_mbarrier_init_cluster();
+    }
+    // activation rows n >= B of every stage stay zero: the consumers load
+    // all 8 rows without a branch
+    for (int i = threadIdx.x; i < stages * 8 * 8 * 4; i += blockDim.x) {
+        const int s = i / (8 * 8 * 4);
+        const int slot = (i / 32) % 8;
+        const int n = (i / 4) % 8;
+        const int t = i % 4;
+        if (n >= B)
+            *reinterpret_cast<uint4*>(smem + geo.stage_bytes * s + geo.off_xp +
+                                      ((slot * 8 + n) * 4 + t) * 16) = make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+    grid_launch_dependents();
+
+    if (warp == CW) {
+        // ------------------------------------------------------ producer
+        if (lane == 0 && nit > 0) {
+            prefetch_tmap(&tmap_w);
+            prefetch_tmap(&tmap_x);
+            const uint32_t tx = RT * kChunkBytes + B * 512 +
+                                (meta_tma ? RT * 16 * (SYM ? 1 : 2) : 0);
+            // weights and scales of the first stages before the dependency wait
+            const int pre = nit < stages ? nit : stages;
+            {
+                int tile = tile0, chunk = chunk0;
+                for (int c = 0; c < pre; ++c) {
+                    uint8_t* st = smem + geo.stage_bytes * c;
+                    mbar_arrive_expect_tx(&full[c], tx);
+                    tma_load_2d(st, &tmap_w, chunk * kChunkBytes, tile * RT, &full[c]);
+                    if (meta_tma) {
+                        const int win = (chunk * GPC) & ~7;
+                        tma_load_2d(st + geo.off_sc, &tmap_s, win, tile * RT, &full[c]);
+                        if constexpr (!SYM) tma_load_2d(st + geo.off_zc, &tmap_z, win, tile * RT, &full[c]);
+                    }
+                    if (++chunk == nchunks) {
+                        chunk = 0;
+                        ++tile;
+                    }
+                }
+            }
+            grid_dependency_wait();
+            bool ok = true;
+            int tile = tile0, chunk = chunk0, s = 0;
+            uint32_t ph = 0;
+            for (int c = 0; c < nit && ok; ++c) {
+                if (c >= stages) ok = mbar_wait_bounded(&empty[s], ph ^ 1u, status, kWaitLimitNs);
+                if (!ok) break;
+                uint8_t* st = smem + geo.stage_bytes * s;
+                if (c >= pre) {
+                    mbar_arrive_expect_tx(&full[s], tx);
+                    tma_load_2d(st, &tmap_w, chunk * kChunkBytes, tile * RT, &full[s]);
+                    if (meta_tma) {
+                        const int win = (chunk * GPC) & ~7;
+                        tma_load_2d(st + geo.off_sc, &tmap_s, win, tile * RT, &full[s]);
+                        if constexpr (!SYM) tma_load_2d(st + geo.off_zc, &tmap_z, win, tile * RT, &full[s]);
+                    }
+                }
+                tma_load_2d(st + geo.off_x, &tmap_x, chunk * kChunkCodes, 0, &full[s]);
+                if (++chunk == nchunks) {
+                    chunk = 0;
+                    ++tile;
+                }
+                if (++s == stages) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            for (int s2 = 0; s2 < stages && s2 < nit; ++s2) {
+                const int last = s2 + ((nit - 1 - s2) / stages) * stages;
+                mbar_wait_bounded(&full[s2], (last / stages) & 1, status, kWaitLimitNs);
+            }
+        }
+        __syncwarp();
+        return;
+    }
+
+    if (warp == CW + 1) {
+        // --------------------------------------------------------- helper
+        // Lane l owns the 8-value block l of each activation row of a chunk
+        // (256 = 32 x 8): it stores the block pair-permuted at the fragment
+        // slot of the consumer thread that multiplies those codes, and adds
+        // its values; GS/8 consecutive lanes form a group, reduced by
+        // shuffles in a fixed order.
+        const int hgq = lane / (GS / 8);
+        const int rem = lane % (GS / 8);
+        const int ht = rem / WPG;
+        const int hi = rem % WPG;
+        grid_dependency_wait();
+        int tile = tile0, chunk = chunk0, s = 0;
+        uint32_t ph = 0;
+        const uint32_t sbase = smem_u32(smem);
+        const uint32_t sbytes = static_cast<uint32_t>(geo.stage_bytes);
+        const uint32_t oX = static_cast<uint32_t>(geo.off_x), oXP = static_cast<uint32_t>(geo.off_xp);
+        const uint32_t oSX = static_cast<uint32_t>(geo.off_sx);
+        const uint32_t xp_lane = oXP + static_cast<uint32_t>((((hgq * WPG + hi) * 8) * 4 + ht) * 16);
+        for (int c = 0; c < nit; ++c) {
+            if (!mbar_wait_bounded(&full[s], ph, status, kWaitLimitNs)) break;
+            uint8_t* st = smem + geo.stage_bytes * s;
+            const uint32_t sa = sbase + sbytes * static_cast<uint32_t>(s);
+            for (int n = 0; n < B; ++n) {
+                const uint4 q = lds128(sa + oX + n * 512 + lane * 16);
+                uint4 o;
+                o.x = pair_lo(q.x, q.z);  // (x0, x4)
+                o.y = pair_hi(q.x, q.z);  // (x1, x5)
+                o.z = pair_lo(q.y, q.w);  // (x2, x6)
+                o.w = pair_hi(q.y, q.w);  // (x3, x7)
+                sts128(sa + xp_lane + n * 64, o);
+                const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+                float v = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if constexpr (BF16) {
+                        v += __uint_as_float(wv[e] << 16);
+                        v += __uint_as_float(wv[e] & 0xFFFF0000u);
+                    } else {
+                        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[e]));
+                        v += f.x;
+                        v += f.y;
+                    }
+                }
+#pragma unroll
+                for (int off = GS / 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+                if (rem == 0) sts32(sa + oSX + (hgq * 8 + n) * 4, __float_as_uint(v));
+            }
+            // sums of the absent batch rows are zero
+            for (int idx = lane; idx < GPC * 8; idx += 32) {
+                if ((idx & 7) >= B) sts32(sa + oSX + idx * 4, 0u);
+            }
+            if (!meta_tma) {
+                // scales (and zero points) at their places in the window
+                uint16_t* scs = reinterpret_cast<uint16_t*>(st + geo.off_sc);
+                uint16_t* zcs = reinterpret_cast<uint16_t*>(st + geo.off_zc);
+                const int64_t g0 = static_cast<int64_t>(chunk) * GPC;
+                const int wofs = (chunk * GPC) & 7;
+                for (int idx = lane; idx < RT * GPC; idx += 32) {
+                    const int r = idx / GPC;
+                    const int gq = idx % GPC;
+                    const int64_t row = static_cast<int64_t>(tile) * RT + r;
+                    const bool okg = row < out && g0 + gq < G;
+                    scs[r * 8 + wofs + gq] = okg ? __ldg(scales + row * G + g0 + gq) : 0;
+                    if constexpr (!SYM) zcs[r * 8 + wofs + gq] = okg ? __ldg(zeros + row * G + g0 + gq) : 0;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sxful[s]);
+            if (++chunk == nchunks) {
+                chunk = 0;
+                ++tile;
+            }
+            if (++s == stages) {
+                s = 0;
+                ph ^= 1u;
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers
+    const int gid = lane >> 2;
+    const int t = lane & 3;
+    const int R0 = warp * 16 + rho(gid);  // rows R0 and R0 + 8 of the tile
+    // byte offset (swizzled) of this thread's words of group gq inside a row
+    int swo[GPC];
+#pragma unroll
+    for (int gq = 0; gq < GPC; ++gq) {
+        const int byte = gq * (GS / 2) + t * (GS / 8);
+        swo[gq] = (((byte >> 4) ^ (R0 & 7)) << 4) | (byte & 15);
+    }
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    int seg_start = 0;  // first iteration (relative) of the current segment
+    int cur_tile = tile0, cur_chunk = chunk0, s = 0;
+    uint32_t ph = 0;
+    grid_dependency_wait();  // y and the workspace are written below
+
+    // 32-bit shared addresses of this thread's loads inside a stage
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sbytes = static_cast<uint32_t>(geo.stage_bytes);
+    const uint32_t a_xp = static_cast<uint32_t>(geo.off_xp) + (gid * 4 + t) * 16;
+    const uint32_t a_sx = static_cast<uint32_t>(geo.off_sx) + 2 * t * 4;
+    const uint32_t a_sc0 = static_cast<uint32_t>(geo.off_sc) + R0 * 16;
+    const uint32_t a_zc0 = static_cast<uint32_t>(geo.off_zc) + R0 * 16;
+    uint32_t a_w[GPC];
+#pragma unroll
+    for (int gq = 0; gq < GPC; ++gq) a_w[gq] = R0 * kChunkBytes + swo[gq];
+
+    bool ok = true;
+    for (int c = 0; c < nit; ++c) {
+        if (ok) ok = mbar_wait_bounded(&full[s], ph, status, kWaitLimitNs);
+        if (ok) ok = mbar_wait_bounded(&sxful[s], ph, status, kWaitLimitNs);
+        if (ok) {
+            const uint32_t sa = sbase + sbytes * static_cast<uint32_t>(s);
+            const uint32_t wofs2 = ((cur_chunk * GPC) & 7) * 2;  // byte offset in the window
+#pragma unroll
+            for (int gq = 0; gq < GPC; ++gq) {
+                uint32_t xf[WPG][4];
+#pragma unroll
+                for (int i = 0; i < WPG; ++i) {
+                    const uint4 v = lds128(sa + a_xp + (gq * WPG + i) * 8 * 64);
+                    xf[i][0] = v.x;
+                    xf[i][1] = v.y;
+                    xf[i][2] = v.z;
+                    xf[i][3] = v.w;
+                }
+                uint32_t w0[WPG], w1[WPG];
+                const uint32_t p0 = sa + a_w[gq];
+                const uint32_t p1 = p0 + 8 * kChunkBytes;
+                if constexpr (WPG == 4) {
+                    const uint4 a = lds128(p0);
+                    const uint4 b = lds128(p1);
+                    w0[0] = a.x; w0[1] = a.y; w0[2] = a.z; w0[3] = a.w;
+                    w1[0] = b.x; w1[1] = b.y; w1[2] = b.z; w1[3] = b.w;
+                } else if constexpr (WPG == 2) {
+                    const uint2 a = lds64(p0);
+                    const uint2 b = lds64(p1);
+                    w0[0] = a.x; w0[1] = a.y;
+                    w1[0] = b.x; w1[1] = b.y;
+                } else {
+                    w0[0] = lds32(p0);
+                    w1[0] = lds32(p1);
+                }
+                float pa[4] = {0.f, 0.f, 0.f, 0.f};
+                float pb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int i = 0; i < WPG; ++i) {
+                    const uint32_t a = w0[i], b = w1[i];
+                    const uint32_t A0[4] = {lop3_and_xor(a, 0x000F000Fu, kMagic),
+                                            lop3_and_xor(b, 0x000F000Fu, kMagic),
+                                            lop3_and_xor(shr_fma<4>(a), 0x000F000Fu, kMagic),
+                                            lop3_and_xor(shr_fma<4>(b), 0x000F000Fu, kMagic)};
+                    const uint32_t A1[4] = {lop3_and_xor(shr_fma<8>(a), 0x000F000Fu, kMagic),
+                                            lop3_and_xor(shr_fma<8>(b), 0x000F000Fu, kMagic),
+                                            lop3_and_xor(shr_fma<12>(a), 0x000F000Fu, kMagic),
+                                            lop3_and_xor(shr_fma<12>(b), 0x000F000Fu, kMagic)};
+                    mma_16816<BF16>(pa, A0, xf[i][0], xf[i][1]);
+                    mma_16816<BF16>(pb, A1, xf[i][2], xf[i][3]);
+                }
+                const uint2 sxw = lds64(sa + a_sx + gq * 32);
+                const float2 sxv = make_float2(__uint_as_float(sxw.x), __uint_as_float(sxw.y));
+                const float s0 = __half2float(__ushort_as_half(lds16(sa + a_sc0 + wofs2 + gq * 2)));
+                const float s1 = __half2float(__ushort_as_half(lds16(sa + a_sc0 + 128 + wofs2 + gq * 2)));
+                float c0, c1;
+                if constexpr (SYM) {
+                    c0 = c1 = Magic<BF16>::base + 8.0f;
+                } else {
+                    c0 = Magic<BF16>::base + __half2float(__ushort_as_half(lds16(sa + a_zc0 + wofs2 + gq * 2)));
+                    c1 = Magic<BF16>::base + __half2float(__ushort_as_half(lds16(sa + a_zc0 + 128 + wofs2 + gq * 2)));
+                }
+                acc[0] = fmaf(s0, fmaf(-c0, sxv.x, pa[0] + pb[0]), acc[0]);
+                acc[1] = fmaf(s0, fmaf(-c0, sxv.y, pa[1] + pb[1]), acc[1]);
+                acc[2] = fmaf(s1, fmaf(-c1, sxv.x, pa[2] + pb[2]), acc[2]);
+                acc[3] = fmaf(s1, fmaf(-c1, sxv.y, pa[3] + pb[3]), acc[3]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+
+        // ---------------------------------------------- segment epilogue
+        if (cur_chunk == nchunks - 1 || c == nit - 1) {
+            const int64_t tile = cur_tile;
+            const int64_t row0 = tile * RT;
+            const bool whole = (c - seg_start) == cur_chunk && cur_chunk == nchunks - 1;
+            if (whole) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int col = 2 * t + (e & 1);
+                    const int64_t row = row0 + R0 + ((e >> 1) ? 8 : 0);
+                    if (col < B && row < out) store_y(y, ydt, static_cast<int64_t>(col) * out + row, acc[e]);
+                }
+            } else {
+                // partial tile: slot 2p (the range's first segment) or 2p + 1
+                const int slot = static_cast<int>(2 * p + (seg_start == 0 ? 0 : 1));
+                float* part = ws_part + static_cast<size_t>(slot) * RT * 8;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int col = 2 * t + (e & 1);
+                    const int row = R0 + ((e >> 1) ? 8 : 0);
+                    __stcg(part + row * 8 + col, acc[e]);
+                }
+                const int64_t q_lo = sk_owner(tile * nchunks, T, P);
+                const int64_t q_hi = sk_owner(tile * nchunks + nchunks - 1, T, P);
+                // one release-acquire atomic per CTA, after the barrier that
+                // orders every consumer's partial stores before it
+                named_bar_sync(1, CW * 32);
+                if (threadIdx.x == 0) {
+                    const unsigned prev = atom_add_acq_rel_gpu(ws_count + tile, 1u);
+                    const bool last = prev == static_cast<unsigned>(q_hi - q_lo);
+                    *last_flag = last ? 1u : 0u;
+                    if (last) ws_count[tile] = 0u;  // zero again for the next call
+                }
+                named_bar_sync(1, CW * 32);
+                if (*last_flag) {
+                    float sum[4] = {0.f, 0.f, 0.f, 0.f};
+                    // contributors in CTA order; 8 loads issued before their adds
+                    for (int64_t q0 = q_lo; q0 <= q_hi; q0 += 8) {
+                        float v[8][4];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int64_t q = q0 + u;
+                            const bool live = q <= q_hi;
+                            const bool first_seg = (T * q) / P >= tile * nchunks;
+                            const int qs = static_cast<int>(2 * q + (first_seg ? 0 : 1));
+                            const float* pq = ws_part + static_cast<size_t>(live ? qs : 0) * RT * 8;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int col = 2 * t + (e & 1);
+                                const int row = R0 + ((e >> 1) ? 8 : 0);
+                                v[u][e] = live ? __ldcg(pq + row * 8 + col) : 0.f;
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) sum[e] += v[u][e];
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int col = 2 * t + (e & 1);
+                        const int64_t row = row0 + R0 + ((e >> 1) ? 8 : 0);
+                        if (col < B && row < out) store_y(y, ydt, static_cast<int64_t>(col) * out + row, sum[e]);
+                    }
+                }
+                named_bar_sync(1, CW * 32);
+            }
+            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+            seg_start = c + 1;
+        }
+        if (++cur_chunk == nchunks) {
+            cur_chunk = 0;
+            ++cur_tile;
+        }
+        if (++s == stages) {
+            s = 0;
+            ph ^= 1u;
+        }
+    }
+}
+
+}  // namespace q4dev

@@ -98,9 +98,9 @@ def test_quantize_pack_validation(lib):
 
 def test_product_validation(lib):
     for fn, bmax in ((lib.q4_gemv, 8), (lib.q4_gemm_skinny, 128)):
-        def call(w=None, x=A16, xdt=q4.Q4_BF16, B=1, y=A16, ydt=q4.Q4_BF16):
+        def call(w=None, x=A16, xdt=q4.Q4_BF16, B=1, y=A16, ydt=q4.Q4_BF16, ws=None, wsb=0):
             w = w if w is not None else _w()
-            return fn(ctypes.byref(w), x, xdt, B, y, ydt, None)
+            return fn(ctypes.byref(w), x, xdt, B, y, ydt, ws, wsb, None)
 
         assert call(B=0) == q4.Q4_ERR_SHAPE
         assert call(B=bmax + 1) == q4.Q4_ERR_SHAPE
@@ -120,6 +120,7 @@ def test_product_validation(lib):
         assert call(w=_w(qweight=A2)) == q4.Q4_ERR_ALIGNMENT
         assert call(w=_w(scales=A16 + 1)) == q4.Q4_ERR_ALIGNMENT
         assert call(w=_w(out=0)) == q4.Q4_OK
+        assert call() == q4.Q4_ERR_WORKSPACE            # no workspace given
 
 
 def test_bf16_reference_and_dequant_validation(lib):
@@ -136,6 +137,13 @@ def test_bf16_reference_and_dequant_validation(lib):
     assert d(ctypes.byref(_w()), A2, q4.Q4_F32, None) == q4.Q4_ERR_ALIGNMENT
     assert d(None, A16, q4.Q4_F32, None) == q4.Q4_ERR_INVALID_ARG
     assert d(ctypes.byref(_w(bits=2)), A16, q4.Q4_F32, None) == q4.Q4_ERR_UNSUPPORTED
+
+
+def test_workspace_query(lib):
+    assert lib.q4_workspace_bytes(0, 256, 1, 128) == 0
+    assert lib.q4_workspace_bytes(64, 0, 1, 128) == 0
+    assert lib.q4_workspace_bytes(64, 256, 0, 128) == 0
+    assert lib.q4_workspace_bytes(64, 256, 129, 128) == 0
 
 
 def test_selftest_validation(lib):

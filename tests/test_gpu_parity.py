@@ -276,3 +276,41 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert q4.q4_sync_status() == q4.Q4_ERR_TIMEOUT
     assert q4.q4_sync_status() == q4.Q4_OK                      # cleared
     _gemv_case(256, 1024, 128, True, 2, torch.bfloat16)          # still usable
+
+
+def test_workspace_contract():
+    """Every completed call leaves the workspace's counters (its last bytes,
+    one per 128-row tile, padded to 256 bytes) at zero; a short workspace is
+    rejected; results do not depend on the buffer's previous contents."""
+    W = wl.normal_weight(3000, 4096, 12, device="cuda")
+    w = q4.q4_quantize_pack(W, 128, True)
+    x = wl.activations(3, 4096, 13, device="cuda")
+    need = q4.load_library().q4_workspace_bytes(w.out, w.in_features, 3, 128)
+    assert need > 0
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    y1 = q4.q4_gemv(w, x, y_dtype=torch.float32, workspace=ws)
+    torch.cuda.synchronize()
+    assert not ws[-256:].any()
+    y2 = q4.q4_gemv(w, x, y_dtype=torch.float32, workspace=ws)
+    assert not ws[-256:].any()
+    assert torch.equal(y1, y2)
+    with pytest.raises(q4.Q4Error) as e:
+        q4.q4_gemv(w, x, workspace=ws[: need - 256])
+    assert e.value.status == q4.Q4_ERR_WORKSPACE
+
+
+def test_workspace_shared_across_shapes():
+    """One buffer serves calls of different shapes in any order: a call with
+    few row tiles leaves partial sums where a larger call keeps counters only
+    if the layout depended on the shape."""
+    big = (28672, 8192)
+    need = q4.load_library().q4_workspace_bytes(big[0], big[1], 4, 128)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for (out, inn) in [(300, 4096), (4096, 4096), big, (1000, 8192), big]:
+        W = wl.normal_weight(out, inn, out, device="cuda")
+        w = q4.q4_quantize_pack(W, 128, True)
+        x = wl.activations(4, inn, 7, device="cuda")
+        y = q4.q4_gemv(w, x, y_dtype=torch.float32, workspace=ws)
+        ref = x.float() @ q4.q4_dequant(w, torch.float32).T
+        rms = ref.pow(2).mean().sqrt()
+        assert torch.all((y - ref).abs() <= 4e-3 * (ref.abs() + rms)), (out, inn)
