@@ -8,7 +8,7 @@ fp16 generated on the device from seeds, quantized with q4_quantize_pack and
 the fp16 copies freed; activations are bf16 N(0, 1).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload llama3-8b | llama3-70b-stack | sweep]
+                    [--workload llama3-8b] [--layers L] [--no-cpu-baseline]
 
 Prints one JSON line (rank 0).  ``value`` is the aggregate HBM throughput of
 the INT4 products (algorithmic bytes / device time, CUDA events, max over
@@ -34,6 +34,15 @@ METRIC = "W4A16 GEMV µs/layer + HBM GB/s (% of B200 peak) at B=1; INT4/bf16 spe
 UNIT = "GB/s"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# DRAM traffic of q4_gemv_sk_kernel per algorithmic byte, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum = 30.33 MB on a 14336 x 4096
+# gate_proj launch whose algorithmic bytes are 30.28 MB).  Scaled to the
+# bench's average launch; it must be re-taken whenever the kernel changes.
+GEMV_TRAFFIC_RATIO = 30.33 / 30.28
+GEMV_TRAFFIC_SOURCE = ("ncu --set full on one 14336x4096 B=1 launch "
+                       "(profiles/q4_gemv_sk_llama3_8b_gate_full.txt), scaled by algorithmic bytes")
 
 
 def load_peaks():
@@ -296,8 +305,11 @@ def run_ours(args):
                           "us_per_layer": round(ms_q * 1e3, 2)},
         "roofline": {"bound": "hbm", "achieved": round(value / world, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(value / world / peak, 4),
-                     "peak_kind": peak_kind, "traffic": None,
-                     "kernel": "q4_gemv_kernel<bf16,g128,sym>",
+                     "peak_kind": peak_kind,
+                     "traffic": round(step_bytes / launches_per_step * GEMV_TRAFFIC_RATIO),
+                     "traffic_unit": "DRAM bytes per launch",
+                     "traffic_source": GEMV_TRAFFIC_SOURCE,
+                     "kernel": "q4_gemv_sk_kernel<bf16,g128,sym,8>",
                      "bytes_per_launch_avg": step_bytes // launches_per_step},
         "clocks": clocks,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
