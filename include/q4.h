@@ -169,6 +169,42 @@ Q4_API q4_status q4_gemm_skinny(const q4_weight* w, const void* x, q4_dtype x_dt
                                 size_t workspace_bytes, q4_stream stream);
 
 /*
+ * Size of the static device scratch that q4_gemv_noalloc uses (3 MiB): it
+ * covers every shape q4_gemv accepts on a GPU with up to 176 SMs.
+ */
+#define Q4_NOALLOC_SCRATCH_BYTES (3u << 20)
+
+/*
+ * q4_gemv without a caller workspace and without any allocation.  The
+ * method's papers have no counterpart to this entry point: it is a
+ * deployment variant for callers that cannot allocate device memory at call
+ * time -- a serving engine that reserved nearly all free HBM for its KV cache
+ * at start-up (a later cudaMalloc fails), a caller that must not pay the
+ * device-wide synchronisation that cudaFree implies inside a decode loop,
+ * and plain C hosts with no allocator to hand the library.
+ *
+ * Arguments, layouts, result and tolerance are those of q4_gemv (1 <= B <= 8).
+ * The stream-K scratch (partial sums and per-row-tile counters) lives in a
+ * static __device__ array of Q4_NOALLOC_SCRATCH_BYTES inside the library;
+ * a shape whose scratch (q4_workspace_bytes) exceeds that returns
+ * Q4_ERR_WORKSPACE before anything is launched.  No device memory is
+ * allocated or freed, by the library or by anything it calls.
+ *
+ * The first call on each device does setup: with that device current it
+ * looks up the scratch address (a failure returns Q4_ERR_CUDA), zero-fills
+ * the scratch on `stream` and waits for that stream.  Make the first call
+ * before any stream capture.  Completed calls leave the counters at zero;
+ * after q4_sync_status has reported Q4_ERR_TIMEOUT the next call zero-fills
+ * the scratch again on its stream before launching.
+ *
+ * All calls on one device share the one scratch: calls that may overlap on
+ * the GPU (different streams, or different host threads without ordering)
+ * race on it and give wrong results.  Issue them in one stream order.
+ */
+Q4_API q4_status q4_gemv_noalloc(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B,
+                                 void* y, q4_dtype y_dtype, q4_stream stream);
+
+/*
  * The unquantised bf16 product y = x W^T with fp32 accumulation, the
  * baseline the INT4 path is compared against and the probe of the bandwidth
  * a weight stream reaches (ybb.press section 一, roofline_bound; arganzheng.

@@ -36,7 +36,7 @@ _DT = {torch.float16: Q4_F16, torch.bfloat16: Q4_BF16, torch.float32: Q4_F32}
 ABI_SYMBOLS = (
     "q4_quantize_pack", "q4_dequant", "q4_gemv", "q4_gemm_skinny", "bf16_gemv_ref_bw",
     "q4_sync_status", "q4_status_string", "q4_version", "q4_selftest_wait_timeout",
-    "q4_workspace_bytes",
+    "q4_workspace_bytes", "q4_gemv_noalloc",
 )
 
 
@@ -84,12 +84,13 @@ def load_library(path: str = LIB_PATH):
     lib.q4_dequant.argtypes = [W, P, S, P]
     lib.q4_gemv.argtypes = [W, P, S, I64, P, S, P, ctypes.c_size_t, P]
     lib.q4_gemm_skinny.argtypes = [W, P, S, I64, P, S, P, ctypes.c_size_t, P]
+    lib.q4_gemv_noalloc.argtypes = [W, P, S, I64, P, S, P]
     lib.q4_workspace_bytes.argtypes = [I64, I64, I64, I32]
     lib.q4_workspace_bytes.restype = ctypes.c_size_t
     lib.bf16_gemv_ref_bw.argtypes = [P, I64, I64, P, I64, P, P]
     lib.q4_sync_status.argtypes = [P]
     lib.q4_selftest_wait_timeout.argtypes = [I64, P]
-    for f in ("q4_quantize_pack", "q4_dequant", "q4_gemv", "q4_gemm_skinny",
+    for f in ("q4_quantize_pack", "q4_dequant", "q4_gemv", "q4_gemm_skinny", "q4_gemv_noalloc",
               "bf16_gemv_ref_bw", "q4_sync_status", "q4_selftest_wait_timeout"):
         getattr(lib, f).restype = S
     lib.q4_status_string.argtypes = [S]
@@ -233,6 +234,25 @@ def q4_gemm_skinny(w: Q4Weight, x: torch.Tensor, y: torch.Tensor | None = None, 
                    workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """y = x W_hat^T for B <= 128."""
     return _product("q4_gemm_skinny", w, x, y, y_dtype, workspace, stream)
+
+
+def q4_gemv_noalloc(w: Q4Weight, x: torch.Tensor, y: torch.Tensor | None = None, y_dtype=None,
+                    stream=None) -> torch.Tensor:
+    """q4_gemv with the library's static device scratch instead of a
+    workspace (B <= 8).  The C call allocates nothing; pass ``y`` to keep
+    this binding from allocating the output.  Calls that may overlap on the
+    GPU race on the one scratch per device."""
+    lib = load_library()
+    if x.dim() != 2:
+        raise ValueError("x must be [B, in]")
+    B = x.shape[0]
+    if y is None:
+        y = torch.empty(B, w.out, dtype=y_dtype or x.dtype, device=x.device)
+    cw = w.c_struct()
+    st = lib.q4_gemv_noalloc(ctypes.byref(cw), _ptr(x), _DT[x.dtype], B, _ptr(y), _DT[y.dtype],
+                             _stream(stream))
+    _check(st, "q4_gemv_noalloc")
+    return y
 
 
 def bf16_gemv_ref_bw(W: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None,

@@ -363,6 +363,51 @@ q4_status validate_product(const q4_weight* w, const void* x, q4_dtype x_dtype, 
     return Q4_OK;
 }
 
+// ------------------------------------------- static scratch (no allocation)
+constexpr size_t kNoAllocScratchBytes = Q4_NOALLOC_SCRATCH_BYTES;
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices];      // scratch address per device, once set up
+bool g_noalloc_reclear[kMaxDevices];   // zero-fill again before the next call
+
+}  // namespace
+
+// Stream-K scratch of q4_gemv_noalloc: partial sums and per-row-tile
+// counters, the same layout as a q4_gemv workspace.  Zero at module load and
+// zero-filled again at setup; the counters must start at zero.
+static __device__ __align__(256) unsigned char g_q4_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Scratch address on the current device `dev`, set up on first use: the
+// symbol address is looked up with `dev` current and the scratch zero-filled
+// on `st`, then `st` is waited for.
+q4_status noalloc_scratch(int dev, cudaStream_t st, void** out) {
+    if (dev < 0 || dev >= kMaxDevices) return Q4_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_q4_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return Q4_ERR_CUDA;
+        if (cudaMemsetAsync(p, 0, kNoAllocScratchBytes, st) != cudaSuccess) return Q4_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return Q4_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+        g_noalloc_reclear[dev] = false;
+    } else if (g_noalloc_reclear[dev]) {
+        if (cudaMemsetAsync(g_noalloc_ptr[dev], 0, kNoAllocScratchBytes, st) != cudaSuccess)
+            return Q4_ERR_CUDA;
+        g_noalloc_reclear[dev] = false;
+    }
+    *out = g_noalloc_ptr[dev];
+    return Q4_OK;
+}
+
+// A bounded wait ran out: counters in the static scratch may be left set.
+void noalloc_mark_reclear() {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    for (int d = 0; d < kMaxDevices; ++d) g_noalloc_reclear[d] = g_noalloc_ptr[d] != nullptr;
+}
+
 }  // namespace
 
 // ======================================================================= ABI
@@ -482,6 +527,24 @@ q4_status q4_gemm_skinny(const q4_weight* w, const void* x, q4_dtype x_dtype, in
     return Q4_ERR_UNSUPPORTED;
 }
 
+q4_status q4_gemv_noalloc(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B,
+                          void* y, q4_dtype y_dtype, q4_stream stream) {
+    q4_status s = validate_product(w, x, x_dtype, B, y, y_dtype, 8);
+    if (s != Q4_OK) return s;
+    if (w->out == 0) return Q4_OK;
+    const int dev = current_device();
+    if (sk_plan(w->out, w->in, sm_count(dev)).ws_bytes > kNoAllocScratchBytes)
+        return Q4_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    void* scratch = nullptr;
+    s = noalloc_scratch(dev, st, &scratch);
+    if (s != Q4_OK) return s;
+    const int ydt = y_dtype == Q4_F32 ? 2 : (y_dtype == Q4_BF16 ? 1 : 0);
+    return x_dtype == Q4_BF16
+               ? dispatch_gemv<true>(w, x, B, y, ydt, scratch, kNoAllocScratchBytes, st)
+               : dispatch_gemv<false>(w, x, B, y, ydt, scratch, kNoAllocScratchBytes, st);
+}
+
 q4_status bf16_gemv_ref_bw(const void* W, int64_t out, int64_t in, const void* x, int64_t B,
                            void* y, q4_stream stream) {
     if (out < 0 || in <= 0 || (in % 64) != 0) return Q4_ERR_SHAPE;
@@ -537,7 +600,10 @@ q4_status q4_sync_status(q4_stream stream) {
         const unsigned zero = 0;
         if (cudaMemcpyToSymbol(g_q4_status, &zero, sizeof(zero)) != cudaSuccess)
             return Q4_ERR_CUDA;
-        if (h & kStatusTimeout) return Q4_ERR_TIMEOUT;
+        if (h & kStatusTimeout) {
+            noalloc_mark_reclear();
+            return Q4_ERR_TIMEOUT;
+        }
     }
     return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
