@@ -157,6 +157,18 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
                  : "r"(a));
     return v;
 }
+// lds128 by the threads with `on` set; the others get zeros and put no
+// request on the shared-memory pipe.
+__device__ __forceinline__ uint4 lds128_if(uint32_t a, bool on) {
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.u32 p, %5, 0;\n\t"
+        "@p ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n\t}"
+        : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w)
+        : "r"(a), "r"(static_cast<uint32_t>(on)));
+    return v;
+}
 __device__ __forceinline__ uint2 lds64(uint32_t a) {
     uint2 v;
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));

@@ -305,6 +305,9 @@ __global__ void __launch_bounds__((CW + 2) * 32, 2)
         const int byte = gq * (GS / 2) + t * (GS / 8);
         swo[gq] = (((byte >> 4) ^ (R0 & 7)) << 4) | (byte & 15);
     }
+    // batch columns n >= B are zero: their threads skip the activation loads
+    // (shared-memory bandwidth, not arithmetic, bounds this loop)
+    const bool x_live = gid < B;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     int seg_start = 0;  // first iteration (relative) of the current segment
     int cur_tile = tile0, cur_chunk = chunk0, s = 0;
@@ -334,7 +337,7 @@ __global__ void __launch_bounds__((CW + 2) * 32, 2)
                 uint32_t xf[WPG][4];
 #pragma unroll
                 for (int i = 0; i < WPG; ++i) {
-                    const uint4 v = lds128(sa + a_xp + (gq * WPG + i) * 8 * 64);
+                    const uint4 v = lds128_if(sa + a_xp + (gq * WPG + i) * 8 * 64, x_live);
                     xf[i][0] = v.x;
                     xf[i][1] = v.y;
                     xf[i][2] = v.z;
