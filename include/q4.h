@@ -123,7 +123,9 @@ Q4_API q4_status q4_dequant(const q4_weight* w, void* W_hat, q4_dtype out_dtype,
 /*
  * Bytes of device workspace that q4_gemv / q4_gemm_skinny need for a weight
  * of this shape and a batch B, on the current device (an upper bound that
- * depends on the device's SM count).  0 for invalid arguments.
+ * depends on the device's SM count and on B).  0 for invalid arguments.
+ * Layout, the same for every shape, batch and kernel: 256 KiB of per-row-tile
+ * counters, then fp32 partial sums.
  */
 Q4_API size_t q4_workspace_bytes(int64_t out, int64_t in, int64_t B, int32_t group_size);
 
@@ -161,8 +163,12 @@ Q4_API q4_status q4_gemv(const q4_weight* w, const void* x, q4_dtype x_dtype, in
 /*
  * The same product for batches 1 <= B <= 128 (the skinny-GEMM regime of
  * arganzheng.life section 二.4, where W4A16 turns compute-bound near
- * B = ridge / 4).  B <= 8 runs the q4_gemv kernel.  Same arguments and
- * requirements as q4_gemv.
+ * B = ridge / 4).  B <= 8 runs the q4_gemv kernel; 9 <= B <= 128 runs on the
+ * tcgen05 tensor cores: codes unpacked to exact 16-bit integers in tensor
+ * memory, activations padded to 16/32/64/128 columns, fp32 accumulation per
+ * group, group partials scaled in fp32.  Same arguments and requirements as
+ * q4_gemv (the workspace of q4_workspace_bytes for this B), same tolerance,
+ * bit-for-bit reproducible.
  */
 Q4_API q4_status q4_gemm_skinny(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B,
                                 void* y, q4_dtype y_dtype, void* workspace,

@@ -16,6 +16,7 @@
 #include "q4_gemv.cuh"
 #include "q4_gemv_sk.cuh"
 #include "q4_quant.cuh"
+#include "q4_skinny_tc.cuh"
 
 namespace {
 
@@ -251,28 +252,51 @@ constexpr int kSkRT = kSkCW * 16;
 constexpr int kSkCtasPerSm = 2;
 constexpr int kSkMinIters = 4;
 
-// Workspace layout, the same for every shape on a device so that one buffer
-// can serve calls of any shape: [partial slots of the largest grid]
-// [one counter per row tile].  Counters are reset by every call that uses
-// them; partial slots never overlap counters.
+// Workspace layout, the same for every shape, batch and kernel so that one
+// buffer can serve any sequence of calls: [one counter per row tile, at most
+// 65535 tiles: kWsCounterBytes] [partial slots of the launch's grid].
+// Counters are reset by every call that uses them; partial slots never
+// overlap counters.
+constexpr size_t kWsCounterBytes = static_cast<size_t>(65536) * 4;
+
 struct SkPlan {
     int64_t row_tiles, T, P;
     int nchunks;
     size_t ws_part_bytes, ws_bytes;
 };
 
-SkPlan sk_plan(int64_t out, int64_t in, int sms) {
+// Stream-K plan over row tiles of `rt` rows and 256-code chunks: at least
+// `min_iters` iterations per CTA (tiny problems use fewer SMs rather than
+// paying a fixup for every chunk), at most `pmax` CTAs; each CTA has two
+// partial slots of rt x `cols` fp32.
+SkPlan stream_k_plan(int64_t out, int64_t in, int rt, int64_t pmax, int min_iters, int cols) {
     SkPlan p{};
-    const int64_t pmax = static_cast<int64_t>(kSkCtasPerSm) * sms;
     p.nchunks = static_cast<int>((in + kChunkCodes - 1) / kChunkCodes);
-    p.row_tiles = (out + kSkRT - 1) / kSkRT;
+    p.row_tiles = (out + rt - 1) / rt;
     p.T = p.row_tiles * p.nchunks;
-    // at least kSkMinIters iterations per CTA: tiny problems use fewer SMs
-    // rather than paying a fixup for every chunk
-    p.P = std::min<int64_t>(std::max<int64_t>(1, p.T / kSkMinIters), pmax);
-    p.ws_part_bytes = static_cast<size_t>(2 * pmax) * kSkRT * 8 * 4;
-    p.ws_bytes = p.ws_part_bytes + align_up(static_cast<size_t>(p.row_tiles) * 4, 256);
+    p.P = std::min<int64_t>(std::max<int64_t>(1, p.T / min_iters), pmax);
+    p.ws_part_bytes = static_cast<size_t>(2 * pmax) * rt * cols * 4;
+    p.ws_bytes = kWsCounterBytes + p.ws_part_bytes;
     return p;
+}
+
+SkPlan sk_plan(int64_t out, int64_t in, int sms) {
+    return stream_k_plan(out, in, kSkRT, static_cast<int64_t>(kSkCtasPerSm) * sms, kSkMinIters, 8);
+}
+
+// Skinny-GEMM (tcgen05) kernel: activation tile width NT per batch size.
+constexpr int kTcMinIters = 4;
+int tc_nt(int64_t B) { return B <= 16 ? 16 : B <= 32 ? 32 : B <= 64 ? 64 : 128; }
+int tc_ctas_per_sm(int nt) { return nt <= 32 ? 2 : 1; }
+
+SkPlan tc_plan(int64_t out, int64_t in, int64_t B, int sms) {
+    const int nt = tc_nt(B);
+    return stream_k_plan(out, in, kTcRT, static_cast<int64_t>(tc_ctas_per_sm(nt)) * sms,
+                         kTcMinIters, nt);
+}
+
+SkPlan product_plan(int64_t out, int64_t in, int64_t B, int sms) {
+    return B <= 8 ? sk_plan(out, in, sms) : tc_plan(out, in, B, sms);
 }
 
 template <bool BF16, int GS, bool SYM>
@@ -320,8 +344,8 @@ q4_status run_gemv(const q4_weight* w, const void* x, int64_t B, void* y, int yd
     unsigned* status = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
         return Q4_ERR_CUDA;
-    float* ws_part = reinterpret_cast<float*>(ws);
-    unsigned* ws_count = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(ws) + p.ws_part_bytes);
+    unsigned* ws_count = reinterpret_cast<unsigned*>(ws);
+    float* ws_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kWsCounterBytes);
     return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3((kSkCW + 2) * 32),
                           geo.total, 1, true, st, tmap_w, tmap_x, tmap_s, tmap_z, meta_tma ? 1 : 0,
                           reinterpret_cast<const uint16_t*>(w->scales),
@@ -342,6 +366,87 @@ q4_status dispatch_gemv(const q4_weight* w, const void* x, int64_t B, void* y, i
         case 128: return sym ? run_gemv<BF16, 128, true>(w, x, B, y, ydt, ws, wsb, st)
                              : run_gemv<BF16, 128, false>(w, x, B, y, ydt, ws, wsb, st);
         default: return Q4_ERR_UNSUPPORTED;
+    }
+}
+
+template <bool BF16, int GS, int NT>
+q4_status run_skinny(const q4_weight* w, const void* x, int64_t B, void* y, int ydt, void* ws,
+                     size_t ws_bytes, cudaStream_t st) {
+    const int dev = current_device();
+    const SkPlan p = tc_plan(w->out, w->in, B, sm_count(dev));
+    if (!ws || ws_bytes < p.ws_bytes) return Q4_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return Q4_ERR_ALIGNMENT;
+    const bool sym = w->symmetric != 0;
+    constexpr int cps = TcCfg<NT>::ctas_per_sm;
+    const size_t per_sm = 228 * 1024;
+    const size_t smax = static_cast<size_t>(max_smem_optin(dev));
+    // deepest ring with `cps` CTAs per SM
+    int stages = kTcMaxStages;
+    TcGeom geo = tc_geom(NT, stages, sym);
+    while (stages > 2 && (cps * (geo.total + 1024) > per_sm || geo.total > smax)) {
+        --stages;
+        geo = tc_geom(NT, stages, sym);
+    }
+    if (cps * (geo.total + 1024) > per_sm || geo.total > smax) return Q4_ERR_UNSUPPORTED;
+    const int64_t G = w->in / GS;
+    const bool meta_tma = (G % 8) == 0 && aligned(w->scales, 16) && (sym || aligned(w->zeros, 16));
+    CUtensorMap tmap_w, tmap_x, tmap_s, tmap_z;
+    std::memset(&tmap_s, 0, sizeof(tmap_s));
+    std::memset(&tmap_z, 0, sizeof(tmap_z));
+    if (!make_tmap_2d(&tmap_w, w->qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                      static_cast<uint64_t>(w->out), static_cast<uint64_t>(w->in / 2), kTcRT,
+                      kChunkBytes))
+        return Q4_ERR_CUDA;
+    // activations: NT-row boxes of 64 values, rows >= B read as zeros
+    if (!make_tmap_2d(&tmap_x, x,
+                      BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                      static_cast<uint64_t>(B), static_cast<uint64_t>(w->in), NT, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+        return Q4_ERR_CUDA;
+    if (meta_tma) {
+        if (!make_tmap_2d(&tmap_s, w->scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                          static_cast<uint64_t>(w->out), static_cast<uint64_t>(G), kTcRT, 8,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+            return Q4_ERR_CUDA;
+        if (!sym && !make_tmap_2d(&tmap_z, w->zeros, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                                  static_cast<uint64_t>(w->out), static_cast<uint64_t>(G), kTcRT,
+                                  8, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return Q4_ERR_CUDA;
+    }
+    auto kernel = q4_skinny_tc_kernel<BF16, GS, NT>;
+    if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), false)) return Q4_ERR_CUDA;
+    unsigned* status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
+        return Q4_ERR_CUDA;
+    unsigned* ws_count = reinterpret_cast<unsigned*>(ws);
+    float* ws_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kWsCounterBytes);
+    return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3(kTcThreads), geo.total, 1, true,
+                     st, tmap_w, tmap_x, tmap_s, tmap_z, meta_tma ? 1 : 0,
+                     reinterpret_cast<const uint16_t*>(w->scales),
+                     reinterpret_cast<const uint16_t*>(w->zeros), sym ? 1 : 0, stages,
+                     static_cast<int>(B), w->out, w->in, p.nchunks, p.T, y, ydt, ws_part, ws_count,
+                     status);
+}
+
+template <bool BF16, int NT>
+q4_status dispatch_skinny_nt(const q4_weight* w, const void* x, int64_t B, void* y, int ydt,
+                             void* ws, size_t wsb, cudaStream_t st) {
+    switch (w->group_size) {
+        case 32: return run_skinny<BF16, 32, NT>(w, x, B, y, ydt, ws, wsb, st);
+        case 64: return run_skinny<BF16, 64, NT>(w, x, B, y, ydt, ws, wsb, st);
+        case 128: return run_skinny<BF16, 128, NT>(w, x, B, y, ydt, ws, wsb, st);
+        default: return Q4_ERR_UNSUPPORTED;
+    }
+}
+
+template <bool BF16>
+q4_status dispatch_skinny(const q4_weight* w, const void* x, int64_t B, void* y, int ydt, void* ws,
+                          size_t wsb, cudaStream_t st) {
+    switch (tc_nt(B)) {
+        case 16: return dispatch_skinny_nt<BF16, 16>(w, x, B, y, ydt, ws, wsb, st);
+        case 32: return dispatch_skinny_nt<BF16, 32>(w, x, B, y, ydt, ws, wsb, st);
+        case 64: return dispatch_skinny_nt<BF16, 64>(w, x, B, y, ydt, ws, wsb, st);
+        default: return dispatch_skinny_nt<BF16, 128>(w, x, B, y, ydt, ws, wsb, st);
     }
 }
 
@@ -502,7 +607,7 @@ q4_status q4_dequant(const q4_weight* w, void* W_hat, q4_dtype out_dtype, q4_str
 size_t q4_workspace_bytes(int64_t out, int64_t in, int64_t B, int32_t group_size) {
     if (out < 0 || in <= 0 || B < 1 || B > 128 || group_size <= 0) return 0;
     if (out == 0) return 0;
-    return sk_plan(out, in, sm_count(current_device())).ws_bytes;
+    return product_plan(out, in, B, sm_count(current_device())).ws_bytes;
 }
 
 q4_status q4_gemv(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B, void* y,
@@ -524,7 +629,13 @@ q4_status q4_gemm_skinny(const q4_weight* w, const void* x, q4_dtype x_dtype, in
     q4_status s = validate_product(w, x, x_dtype, B, y, y_dtype, 128);
     if (s != Q4_OK) return s;
     if (B <= 8) return q4_gemv(w, x, x_dtype, B, y, y_dtype, workspace, workspace_bytes, stream);
-    return Q4_ERR_UNSUPPORTED;
+    if (w->out == 0) return Q4_OK;
+    if (!workspace) return Q4_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int ydt = y_dtype == Q4_F32 ? 2 : (y_dtype == Q4_BF16 ? 1 : 0);
+    return x_dtype == Q4_BF16
+               ? dispatch_skinny<true>(w, x, B, y, ydt, workspace, workspace_bytes, st)
+               : dispatch_skinny<false>(w, x, B, y, ydt, workspace, workspace_bytes, st);
 }
 
 q4_status q4_gemv_noalloc(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B,

@@ -1,0 +1,110 @@
+// q4_tcgen05.cuh -- 5th-generation tensor core (tcgen05) building blocks for
+// sm_100a: tensor-memory allocation, register <-> tensor-memory copies, the
+// shared-memory matrix descriptor of a 128-byte-swizzled K-major tile, the
+// instruction descriptor of a 16-bit MMA with fp32 accumulation, the MMA with
+// its A operand in tensor memory, and completion tracking through mbarriers.
+//
+// Tensor memory (TMEM) is 128 lanes x 512 columns of 32 bits per SM.  An
+// address is (lane << 16) | column; warp w of a CTA may touch only lanes
+// [32 (w % 4), 32 (w % 4) + 32).  An M = 128 accumulator holds row m in lane m;
+// a 16-bit A operand holds row m in lane m with elements k, k+1 packed in one
+// column (k even in the low half).
+#pragma once
+
+#include <stdint.h>
+
+#include "q4_device.cuh"
+
+namespace q4dev {
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Whole-warp TMEM allocation of `ncols` columns (a power of two >= 32); the
+// base address is written to shared memory at `dst`.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// Eight consecutive columns of this thread's lane from / to registers.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+          "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory descriptor of a K-major operand tile stored with the 128-byte
+// swizzle, as a TMA load with CU_TENSOR_MAP_SWIZZLE_128B writes it: rows of
+// 128 bytes, groups of 8 rows 1024 bytes apart, the atom 1024-byte aligned.
+// `saddr` is the shared address of the first row's 16-element (32-byte) K
+// slice; slices further along K inside the 128-byte row are addressed by
+// adding their byte offset to the start address.
+__device__ __forceinline__ uint64_t umma_desc_sw128_kmajor(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);  // start address, 16-byte units
+    d |= static_cast<uint64_t>(16 >> 4) << 16;           // leading offset (unused by SW128 K-major)
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;         // stride between 8-row groups
+    d |= static_cast<uint64_t>(1) << 46;                 // descriptor version of sm_100
+    d |= static_cast<uint64_t>(2) << 61;                 // layout: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: D fp32, A and B bf16 (or fp16), both K-major,
+// M x N with M in {64, 128} and N a multiple of 16 (M = 128).
+template <bool BF16, int M, int N>
+__host__ __device__ constexpr uint32_t umma_idesc_f16() {
+    return (1u << 4) | ((BF16 ? 1u : 0u) << 7) | ((BF16 ? 1u : 0u) << 10) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T for one K = 16 step; `accumulate` = 0
+// overwrites D.  Issued by one thread.
+__device__ __forceinline__ void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
+            tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        : "memory");
+}
+
+// Arrive (once) on `bar` when every MMA this thread issued so far completes.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+}  // namespace q4dev

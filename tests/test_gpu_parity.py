@@ -278,9 +278,12 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     _gemv_case(256, 1024, 128, True, 2, torch.bfloat16)          # still usable
 
 
+WS_COUNTER_BYTES = 65536 * 4  # the workspace starts with one counter per row tile
+
+
 def test_workspace_contract():
-    """Every completed call leaves the workspace's counters (its last bytes,
-    one per 128-row tile, padded to 256 bytes) at zero; a short workspace is
+    """Every completed call leaves the workspace's counters (its first
+    WS_COUNTER_BYTES, one per 128-row tile) at zero; a short workspace is
     rejected; results do not depend on the buffer's previous contents."""
     W = wl.normal_weight(3000, 4096, 12, device="cuda")
     w = q4.q4_quantize_pack(W, 128, True)
@@ -290,9 +293,9 @@ def test_workspace_contract():
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
     y1 = q4.q4_gemv(w, x, y_dtype=torch.float32, workspace=ws)
     torch.cuda.synchronize()
-    assert not ws[-256:].any()
+    assert not ws[:WS_COUNTER_BYTES].any()
     y2 = q4.q4_gemv(w, x, y_dtype=torch.float32, workspace=ws)
-    assert not ws[-256:].any()
+    assert not ws[:WS_COUNTER_BYTES].any()
     assert torch.equal(y1, y2)
     with pytest.raises(q4.Q4Error) as e:
         q4.q4_gemv(w, x, workspace=ws[: need - 256])
@@ -314,3 +317,69 @@ def test_workspace_shared_across_shapes():
         ref = x.float() @ q4.q4_dequant(w, torch.float32).T
         rms = ref.pow(2).mean().sqrt()
         assert torch.all((y - ref).abs() <= 4e-3 * (ref.abs() + rms)), (out, inn)
+
+
+def test_workspace_shared_across_batches():
+    """One buffer, sized for the largest call, serves the small-batch and the
+    tensor-core kernels in any order."""
+    shapes = [(300, 4096, 4), (4096, 4096, 40), (8192, 8192, 2), (1000, 8192, 128), (4096, 4096, 8)]
+    lib = q4.load_library()
+    need = max(lib.q4_workspace_bytes(o, i, b, 128) for o, i, b in shapes)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for (out, inn, B) in shapes:
+        W = wl.normal_weight(out, inn, out + B, device="cuda")
+        w = q4.q4_quantize_pack(W, 128, True)
+        x = wl.activations(B, inn, 7, device="cuda")
+        y = q4.q4_gemm_skinny(w, x, y_dtype=torch.float32, workspace=ws)
+        ref = x.float() @ q4.q4_dequant(w, torch.float32).T
+        rms = ref.pow(2).mean().sqrt()
+        assert torch.all((y - ref).abs() <= 4e-3 * (ref.abs() + rms)), (out, inn, B)
+        torch.cuda.synchronize()
+        assert not ws[:WS_COUNTER_BYTES].any()
+
+
+# ------------------------------------------------- skinny GEMM, 9 <= B <= 128
+
+@pytest.mark.parametrize("xdtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("sym", [True, False])
+@pytest.mark.parametrize("g,inn", [(32, 1120), (64, 1216), (128, 1408)])
+@pytest.mark.parametrize("B", [9, 16, 24, 40, 100, 128])
+def test_skinny_ragged_tiles(xdtype, sym, g, inn, B):
+    # 300 rows = two full 128-row tiles and a ragged third; `in` ends in a
+    # partial 256-code chunk; B pads to the 16/32/64/128-wide MMA tiles
+    _gemv_case(300, inn, g, sym, B, xdtype, api="q4_gemm_skinny")
+
+
+@pytest.mark.parametrize("ydtype", [torch.float32, None])
+@pytest.mark.parametrize("shape,B", [((4096, 4096), 16), ((256, 8192), 32), ((96, 28672), 64),
+                                     ((1024, 4096), 128)])
+def test_skinny_split_k(ydtype, shape, B):
+    # few row tiles and long K: every tile is split across CTAs
+    _gemv_case(*shape, 128, True, B, torch.bfloat16, ydtype=ydtype, api="q4_gemm_skinny")
+
+
+@pytest.mark.parametrize("name", ["q_proj", "gate_proj", "down_proj"])
+@pytest.mark.parametrize("g", [32, 128])
+@pytest.mark.parametrize("B", [16, 64, 128])
+def test_skinny_llama3_70b_heavy_tail(name, g, B):
+    """70B shapes, Student-t(3) weights, 4 outlier activation channels (x20),
+    sampled rows against the oracle."""
+    out, inn = wl.LLAMA3_70B[name]
+    _gemv_case(out, inn, g, True, B, torch.bfloat16, kind="t3", seed=20,
+               rows=_sample_rows(out, 96, seed=B), n_outliers=4, api="q4_gemm_skinny")
+
+
+def test_skinny_consistency():
+    """fp32 and bf16 outputs agree, repeated calls are bit-identical, and the
+    rows of a batched call agree with the same rows run as a batch of 16."""
+    W = wl.normal_weight(700, 2048, 9, device="cuda")
+    x = wl.activations(48, 2048, 10, device="cuda")
+    w = q4.q4_quantize_pack(W, 64, False)
+    y32 = q4.q4_gemm_skinny(w, x, y_dtype=torch.float32)
+    yb = q4.q4_gemm_skinny(w, x)
+    assert torch.equal(y32.to(torch.bfloat16), yb)
+    assert torch.equal(q4.q4_gemm_skinny(w, x, y_dtype=torch.float32), y32)
+    y16 = q4.q4_gemm_skinny(w, x[16:32].contiguous(), y_dtype=torch.float32)
+    ref = x.float() @ q4.q4_dequant(w, torch.float32).T
+    rms = ref.pow(2).mean().sqrt()
+    assert torch.all((y16 - y32[16:32]).abs() <= 4e-3 * (ref[16:32].abs() + rms))
