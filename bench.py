@@ -8,7 +8,8 @@ fp16 generated on the device from seeds, quantized with q4_quantize_pack and
 the fp16 copies freed; activations are bf16 N(0, 1).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload llama3-8b] [--layers L] [--no-cpu-baseline]
+                    [--workload llama3-8b | llama3-70b-stack [--batch B]]
+                    [--layers L] [--no-sweep] [--no-cpu-baseline]
 
 Prints one JSON line (rank 0).  ``value`` is the aggregate HBM throughput of
 the INT4 products (algorithmic bytes / device time, CUDA events, max over
@@ -156,6 +157,64 @@ def time_region(torch, fn, steps, warmup, stream):
     e1.record(stream)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1)  # ms
+
+
+def graph_time_us(torch, fn, n, stream):
+    """Mean device time of one call of fn(i) over n calls captured in a CUDA
+    graph (CUDA events on the launching stream, 2 warm-up replays)."""
+    for i in range(3):
+        fn(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        for i in range(n):
+            fn(i)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    ms = time_region(torch, g.replay, 3, 1, stream)
+    del g
+    return ms * 1e3 / (3 * n)
+
+
+SWEEP_B = (1, 2, 4, 8, 16, 32, 64, 128)
+
+
+def b_sweep(q4, wl, torch, device, stream):
+    """INT4/bf16 speedup vs batch on the Llama-3-70B down_proj shape
+    (8192 x 28672, N(0, 0.02^2), sym g128): q4_gemm_skinny against the bf16
+    product (this library's bf16_gemv_ref_bw for B <= 8, cuBLAS through
+    torch.matmul beyond).  Four INT4 and two bf16 copies rotate so no call
+    finds its weights in L2."""
+    out, inn = wl.LLAMA3_70B["down_proj"]
+    ws = [q4.q4_quantize_pack(wl.normal_weight(out, inn, 30 + i, device=device), 128, True)
+          for i in range(4)]
+    Wb = [wl.normal_weight(out, inn, 40 + i, device=device).to(torch.bfloat16) for i in range(2)]
+    torch.cuda.synchronize()
+    rows = {}
+    for B in SWEEP_B:
+        x = wl.activations(B, inn, 31, device=device)
+        y = torch.empty(B, out, dtype=torch.bfloat16, device=device)
+        wsp = q4.workspace_for(ws[0], B, device)
+        t4 = graph_time_us(torch, lambda i: q4.q4_gemm_skinny(ws[i % 4], x, y=y, workspace=wsp), 16, stream)
+        if B <= 8:
+            tb = graph_time_us(torch, lambda i: q4.bf16_gemv_ref_bw(Wb[i % 2], x, y=y), 16, stream)
+            bf_impl = "bf16_gemv_ref_bw"
+        else:
+            tb = graph_time_us(torch, lambda i: torch.matmul(x, Wb[i % 2].T, out=y), 16, stream)
+            bf_impl = "cublas"
+        rows[B] = {"int4_us": round(t4, 2), "bf16_us": round(tb, 2), "speedup": round(tb / t4, 3),
+                   "int4_gbs": round(algo_bytes(out, inn, 128, B) / t4 / 1e3, 1),
+                   "int4_tflops": round(2 * B * out * inn / t4 / 1e6, 1), "bf16_impl": bf_impl}
+    st = q4.q4_sync_status()
+    assert st == q4.Q4_OK, q4.status_string(st)
+    # knee of max(t_mem, c B): t_mem the B = 1 time, c the B = 128 slope
+    t_mem = rows[1]["int4_us"]
+    c = rows[SWEEP_B[-1]]["int4_us"] / SWEEP_B[-1]
+    even = next((B for B in SWEEP_B if rows[B]["int4_us"] >= rows[B]["bf16_us"]), None)
+    del ws, Wb
+    return {"shape": f"{out}x{inn} sym g128", "by_B": rows, "knee_B": round(t_mem / c, 1),
+            "B_even": even if even is not None else f"> {SWEEP_B[-1]}"}
 
 
 def run_ours(args):
@@ -317,6 +376,8 @@ def run_ours(args):
         "gpu_launches": args.steps * launches_per_step,
     }
     if rank == 0:
+        if world == 1 and not args.no_sweep:
+            out["int4_vs_bf16_by_B"] = b_sweep(q4, wl, torch, device, stream)
         out["cpu_baseline"] = cpu_baseline() if (world == 1 and not args.no_cpu_baseline) else None
         print(json.dumps(out), flush=True)
     del graph
@@ -324,6 +385,96 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
 
+
+
+def run_stack(args):
+    """Llama-3-70B decode stack: 80 distinct layers x 7 linears (560 W4A16
+    products of 34.2 GB of packed weights), asymmetric group 64, batch B, one
+    CUDA graph per step.  Weights N(0, 0.02^2) fp16 generated on the device
+    per layer (seed 1000 layer + linear index), quantized, fp16 freed."""
+    import torch
+
+    import post_weight_quantization_group_b200 as q4
+    from post_weight_quantization_group_b200 import workloads as wl
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    q4.load_library()
+    peaks, peak_kind = load_peaks()
+    stream = torch.cuda.current_stream()
+    B, g = args.batch, 64
+    shapes = wl.LLAMA3_70B
+    mats = []
+    for layer in range(80):
+        for idx, (name, (out, inn)) in enumerate(shapes.items()):
+            W = wl.normal_weight(out, inn, wl.llama3_70b_stack_seed(layer, idx), device=device)
+            mats.append((name, q4.q4_quantize_pack(W, g, False)))
+            del W
+    torch.cuda.synchronize()
+    xs = {inn: wl.activations(B, inn, 17 + inn, device=device) for _, (_, inn) in shapes.items()}
+    ys = {name: torch.empty(B, out, dtype=torch.bfloat16, device=device) for name, (out, _) in shapes.items()}
+    ws = q4.workspace_for(mats[0][1], B, device)
+    for _, w in mats:
+        ws = q4.workspace_for(w, B, device)
+    step_bytes = sum(algo_bytes(*shapes[n], g, B, sym=False) for n, _ in mats)
+
+    def step():
+        for name, w in mats:
+            q4.q4_gemm_skinny(w, xs[shapes[name][1]], y=ys[name], workspace=ws)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    assert q4.q4_sync_status() == q4.Q4_OK
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+        step()
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        ms = time_region(torch, graph.replay, args.steps, args.warmup, stream)
+    st = q4.q4_sync_status()
+    assert st == q4.Q4_OK, q4.status_string(st)
+    value = step_bytes * args.steps / (ms * 1e-3) / 1e9
+    x_host = {k: v.cpu().pin_memory() for k, v in xs.items()}
+    y_host = torch.empty(B, shapes["down_proj"][0], dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step():
+        for k, v in x_host.items():
+            xs[k].copy_(v, non_blocking=True)
+        graph.replay()
+        y_host.copy_(ys["down_proj"], non_blocking=True)
+        stream.synchronize()
+
+    ne = max(3, args.steps // 4)
+    e2e_step()
+    t0 = time.perf_counter()
+    for _ in range(ne):
+        e2e_step()
+    e2e_value = step_bytes * ne / (time.perf_counter() - t0) / 1e9
+    peak = peaks["hbm_gbs"]
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02^2) fp16 weights quantized on device; bf16 N(0,1) activations)",
+        "config": {"workload": f"Llama-3-70B decode stack: 80 layers x q,k,v,o,gate,up,down, asym g64, B={B}",
+                   "batch": B, "group_size": g, "symmetric": False, "layers": 80,
+                   "linears_per_step": len(mats), "bytes_per_step": step_bytes,
+                   "l2": f"inputs larger than L2 ({step_bytes / 1e9:.1f} GB per step)",
+                   "timing": "CUDA graph of the step, CUDA events on the launching stream"},
+        "us_per_layer": round(ms / args.steps / 80 * 1e3, 2),
+        "roofline": {"bound": "hbm", "achieved": round(value, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(value / peak, 4), "peak_kind": peak_kind, "traffic": None,
+                     "kernel": "q4_gemv_sk_kernel" if B <= 8 else "q4_skinny_tc_kernel"},
+        "clocks": clk.summary(),
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT,
+                "h2d_bytes_per_step": sum(v.numel() * v.element_size() for v in x_host.values()),
+                "d2h_bytes_per_step": y_host.numel() * y_host.element_size(), "steps": ne},
+        "gpu_launches": args.steps * len(mats),
+        "cpu_baseline": None,
+    }
+    print(json.dumps(out), flush=True)
+    del graph
 
 # ------------------------------------------------------- CPU oracle timing
 def _oracle_layer():
@@ -414,9 +565,12 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llama3-8b", choices=["llama3-8b"])
+    ap.add_argument("--workload", default="llama3-8b", choices=["llama3-8b", "llama3-70b-stack"])
+    ap.add_argument("--batch", type=int, default=1, help="batch of the llama3-70b-stack workload")
     ap.add_argument("--layers", type=int, default=32,
                     help="distinct decoder layers per step (32 = the Llama-3-8B depth)")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the INT4/bf16 speedup-vs-batch sweep (70B down_proj, B = 1..128)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip timing the CPU oracle (profiling runs)")
     args = ap.parse_args()
@@ -424,6 +578,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "llama3-70b-stack":
+        run_stack(args)
     else:
         run_ours(args)
 

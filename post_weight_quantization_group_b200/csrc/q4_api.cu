@@ -420,7 +420,8 @@ q4_status run_skinny(const q4_weight* w, const void* x, int64_t B, void* y, int 
         return Q4_ERR_CUDA;
     unsigned* ws_count = reinterpret_cast<unsigned*>(ws);
     float* ws_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kWsCounterBytes);
-    return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3(kTcThreads), geo.total, 1, true,
+    return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3(TcCfg<NT>::threads), geo.total,
+                     1, true,
                      st, tmap_w, tmap_x, tmap_s, tmap_z, meta_tma ? 1 : 0,
                      reinterpret_cast<const uint16_t*>(w->scales),
                      reinterpret_cast<const uint16_t*>(w->zeros), sym ? 1 : 0, stages,

@@ -15,17 +15,21 @@
 //    swizzle), of the activations [NT rows x 256] as four 128-byte-swizzled
 //    K-major atoms (rows >= B are filled with zeros by the TMA unit), and of
 //    the scale (and zero-point) window;
-//  * four converter warps, one weight row per thread: each group's codes are
-//    unpacked to exact 16-bit integers q (or q - z) and stored into a tensor
-//    memory A buffer (arganzheng.life post-training-quantization-gptq-awq-
+//  * 4 (NT <= 32) or 16 converter warps, one weight row per thread and
+//    lane, in shares of four warps (one per tensor-memory lane quarter): each
+//    group's codes are unpacked to exact 16-bit integers q (or q - z) and
+//    stored into a tensor-memory A buffer, the 16-byte chunks of a row divided
+//    among the shares (arganzheng.life post-training-quantization-gptq-awq-
 //    and-rotation, section 二.3: the int4 weights are dequantized on chip,
 //    never in HBM);
 //  * MMA warp, one thread: per group, GS/16 tcgen05.mma steps
 //    D[128 x NT] (+)= A[128 x 16] * X[NT x 16]^T into a fresh fp32
 //    accumulator in tensor memory, then a commit;
-//  * the converter warps read each finished group accumulator back and add
-//    it times the group's fp32 scale into registers (section 二.2: per-group
-//    scales are applied inside the K accumulation, one partial per group).
+//  * the converter warps read each finished group accumulator back, each
+//    share its own columns, and add it times the group's fp32 scale into
+//    registers (section 二.2: per-group scales are applied inside the K
+//    accumulation, one partial per group).  The rescale of a group runs one
+//    or two groups after its unpack, so the MMAs overlap the next unpacks.
 //
 // Unpacking keeps K in natural order: for the byte holding codes k and k+1,
 // one PRMT places it and the same byte of the word shifted right by 4 at the
@@ -46,7 +50,6 @@ namespace q4dev {
 
 constexpr int kTcRT = 128;        // rows per tile: MMA M, tensor-memory lanes
 constexpr int kTcMaxStages = 4;
-constexpr int kTcThreads = 192;   // producer, MMA issuer, 4 converter warps
 constexpr int kTcMaxBuf = 4;      // group buffers in tensor memory
 
 template <int NT>
@@ -54,6 +57,13 @@ struct TcCfg {
     // CTAs per SM: tensor memory (512 columns per SM) is split between them
     static constexpr int ctas_per_sm = NT <= 32 ? 2 : 1;
     static constexpr uint32_t tmem_cols = NT <= 32 ? 256u : 512u;
+    // converter warps: H shares of 4 warps (one per tensor-memory lane
+    // quarter); share h unpacks the 16-byte chunks c with c % H == h and
+    // rescales accumulator columns [h NT / H, (h + 1) NT / H).  Narrow tiles
+    // are bound by the MMA rate (one M = 128, K = 16 step takes as long at
+    // N = 16 as at N = 128), wide ones by the rescale work.
+    static constexpr int conv_warps = NT <= 32 ? 4 : 16;
+    static constexpr int threads = (2 + conv_warps) * 32;
 };
 
 struct TcGeom {
@@ -94,7 +104,7 @@ __device__ __forceinline__ void unpack_word_pairs(uint32_t w, uint32_t magic, ui
 }
 
 template <bool BF16, int GS, int NT>
-__global__ void __launch_bounds__(kTcThreads, TcCfg<NT>::ctas_per_sm)
+__global__ void __launch_bounds__(TcCfg<NT>::threads, TcCfg<NT>::ctas_per_sm)
     q4_skinny_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
                         const __grid_constant__ CUtensorMap tmap_x,
                         const __grid_constant__ CUtensorMap tmap_s,
@@ -112,6 +122,11 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<NT>::ctas_per_sm)
     static_assert(NB >= 2, "tensor memory too small for two group buffers");
     constexpr uint32_t kIdesc = umma_idesc_f16<BF16, kTcRT, NT>();
     constexpr uint32_t kDcol0 = NB * ACOLS;    // first accumulator column
+    constexpr int CONV = TcCfg<NT>::conv_warps;
+    constexpr int H = CONV / 4;
+    constexpr int NH = NT / H;                 // accumulator columns per converter warp
+    constexpr int LAG = NB >= 3 ? 2 : 1;       // groups between a group's unpack and its rescale
+    static_assert(NH % 8 == 0, "columns per converter warp");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -140,12 +155,12 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<NT>::ctas_per_sm)
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 5);  // 4 converter warps + the MMA commit
+            mbar_init(&empty[s], CONV + 1);  // converter warps + the MMA commit
         }
         for (int b = 0; b < NB; ++b) {
-            mbar_init(&a_full[b], 4);
+            mbar_init(&a_full[b], CONV);
             mbar_init(&mma_done[b], 1);
-            mbar_init(&acc_free[b], 4);
+            mbar_init(&acc_free[b], CONV);
         }
         mbar_init(drain, 1);
         fence_mbarrier_init_cluster();
@@ -262,17 +277,18 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<NT>::ctas_per_sm)
         }
     } else {
         // ------------------------------------------------------ converters
-        const int q = warp & 3;  // lane quarter of tensor memory
-        const int r = 32 * q + lane;
+        const int q = warp & 3;          // tensor-memory lane quarter (warp % 4)
+        const int h = (warp - 2) >> 2;   // this warp's share of the work
+        const int r = 32 * q + lane;     // weight row of this thread
         const uint32_t tl = tbase + (static_cast<uint32_t>(32 * q) << 16);
         const uint32_t magic = Magic<BF16>::base2 ^ (sym ? 0x00080008u : 0u);
         const uint32_t csym = static_cast<uint32_t>(small_int_bits<BF16>(Magic<BF16>::base + 8.0f)) *
                               0x00010001u;
         grid_dependency_wait();  // y and the workspace are written below
 
-        float yacc[NT];
+        float yacc[NH];
 #pragma unroll
-        for (int n = 0; n < NT; ++n) yacc[n] = 0.f;
+        for (int e = 0; e < NH; ++e) yacc[e] = 0.f;
 
         const uint32_t sbase = smem_u32(smem);
         const uint32_t sbytes = static_cast<uint32_t>(geo.stage_bytes);
@@ -280,78 +296,92 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<NT>::ctas_per_sm)
         int cur_tile = tile0, cur_chunk = chunk0, s = 0, i = 0;
         uint32_t ph = 0;
         int seg_start = 0;
-        // the group waiting for its rescale, and whether it ends a segment
-        float pend_scale = 0.f;
-        bool pend_end = false, pend_whole = false, pend_first = false;
-        int pend_tile = 0;
 
-        // Rescale of group j (accumulator buffer j % NB) and, if it ends a
-        // segment, the segment's epilogue.
-        auto rescale = [&](int j, float sj, bool seg_end, bool whole, bool first_seg, int tile) {
+        // A group waiting for its rescale: its scale and, if it ends a
+        // segment, the segment's tile and kind.
+        struct Pend {
+            float scale;
+            bool end, whole, first;
+            int tile;
+        };
+        Pend p0{0.f, false, false, false, 0}, p1{0.f, false, false, false, 0};
+
+        // Rescale of group j (accumulator buffer j % NB): this warp's NH
+        // columns times the group's scale into yacc; then, if the group ends
+        // a segment, the segment's epilogue.
+        auto rescale = [&](int j, const Pend& pd) {
             const int b = j % NB;
             if (ok) ok = mbar_wait_bounded(&mma_done[b], static_cast<uint32_t>(j / NB) & 1u, status,
                                            kWaitLimitNs);
             tc_fence_after();
             if (ok) {
+                uint32_t v[NH];
 #pragma unroll
-                for (int c0 = 0; c0 < NT; c0 += 16) {
-                    uint32_t v[16];
-                    tmem_ld16(tl + kDcol0 + b * NT + c0, v);
-                    tmem_wait_ld();
+                for (int c0 = 0; c0 < NH; c0 += 8)
+                    tmem_ld8(tl + kDcol0 + b * NT + h * NH + c0,
+                             *reinterpret_cast<uint32_t(*)[8]>(&v[c0]));
+                tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) yacc[c0 + e] = fmaf(sj, __uint_as_float(v[e]), yacc[c0 + e]);
-                }
+                for (int e = 0; e < NH; ++e) yacc[e] = fmaf(pd.scale, __uint_as_float(v[e]), yacc[e]);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_free[b]);
-            if (!seg_end) return;
-            const int64_t row = static_cast<int64_t>(tile) * kTcRT + r;
-            if (whole) {
+            if (!pd.end) return;
+            const int64_t row = static_cast<int64_t>(pd.tile) * kTcRT + r;
+            if (pd.whole) {
                 if (row < out) {
 #pragma unroll
-                    for (int n = 0; n < NT; ++n)
-                        if (n < B) store_y(y, ydt, static_cast<int64_t>(n) * out + row, yacc[n]);
+                    for (int e = 0; e < NH; ++e) {
+                        const int n = h * NH + e;
+                        if (n < B) store_y(y, ydt, static_cast<int64_t>(n) * out + row, yacc[e]);
+                    }
                 }
             } else {
-                const int slot = static_cast<int>(2 * p + (first_seg ? 0 : 1));
+                const int slot = static_cast<int>(2 * p + (pd.first ? 0 : 1));
                 float* part = ws_part + static_cast<size_t>(slot) * kTcRT * NT;
 #pragma unroll
-                for (int n = 0; n < NT; ++n)
-                    if (n < B) __stcg(part + n * kTcRT + r, yacc[n]);
-                const int64_t t64 = tile;
+                for (int e = 0; e < NH; ++e) {
+                    const int n = h * NH + e;
+                    if (n < B) __stcg(part + n * kTcRT + r, yacc[e]);
+                }
+                const int64_t t64 = pd.tile;
                 const int64_t q_lo = sk_owner(t64 * nchunks, T, P);
                 const int64_t q_hi = sk_owner(t64 * nchunks + nchunks - 1, T, P);
-                named_bar_sync(1, 128);
+                named_bar_sync(1, CONV * 32);
                 if (threadIdx.x == 64) {
-                    const unsigned prev = atom_add_acq_rel_gpu(ws_count + tile, 1u);
+                    const unsigned prev = atom_add_acq_rel_gpu(ws_count + pd.tile, 1u);
                     const bool last = prev == static_cast<unsigned>(q_hi - q_lo);
                     *last_flag = last ? 1u : 0u;
-                    if (last) ws_count[tile] = 0u;  // zero again for the next call
+                    if (last) ws_count[pd.tile] = 0u;  // zero again for the next call
                 }
-                named_bar_sync(1, 128);
+                named_bar_sync(1, CONV * 32);
                 if (*last_flag) {
                     // contributors in CTA order
 #pragma unroll
-                    for (int n = 0; n < NT; ++n) yacc[n] = 0.f;
+                    for (int e = 0; e < NH; ++e) yacc[e] = 0.f;
                     for (int64_t qq = q_lo; qq <= q_hi; ++qq) {
                         const bool fs = (T * qq) / P >= t64 * nchunks;
                         const int qs = static_cast<int>(2 * qq + (fs ? 0 : 1));
                         const float* pq = ws_part + static_cast<size_t>(qs) * kTcRT * NT;
 #pragma unroll
-                        for (int n = 0; n < NT; ++n)
-                            if (n < B) yacc[n] += __ldcg(pq + n * kTcRT + r);
+                        for (int e = 0; e < NH; ++e) {
+                            const int n = h * NH + e;
+                            if (n < B) yacc[e] += __ldcg(pq + n * kTcRT + r);
+                        }
                     }
                     if (row < out) {
 #pragma unroll
-                        for (int n = 0; n < NT; ++n)
-                            if (n < B) store_y(y, ydt, static_cast<int64_t>(n) * out + row, yacc[n]);
+                        for (int e = 0; e < NH; ++e) {
+                            const int n = h * NH + e;
+                            if (n < B) store_y(y, ydt, static_cast<int64_t>(n) * out + row, yacc[e]);
+                        }
                     }
                 }
-                named_bar_sync(1, 128);
+                named_bar_sync(1, CONV * 32);
             }
 #pragma unroll
-            for (int n = 0; n < NT; ++n) yacc[n] = 0.f;
+            for (int e = 0; e < NH; ++e) yacc[e] = 0.f;
         };
 
         for (int c = 0; c < nit; ++c) {
@@ -388,6 +418,7 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<NT>::ctas_per_sm)
 #pragma unroll
                     for (int t = 0; t < GS / 32; ++t) {
                         const int c16 = gq * (GS / 32) + t;
+                        if (c16 % H != h) continue;
                         const uint4 w = lds128(sa + r * kChunkBytes + ((c16 ^ (r & 7)) << 4));
                         uint32_t v0[8], v1[8];
                         unpack_word_pairs<BF16>(w.x, magic, c2, v0);
@@ -405,16 +436,20 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<NT>::ctas_per_sm)
                     mbar_arrive(&a_full[b]);
                     if (gq == GPC - 1) mbar_arrive(&empty[s]);  // weights and scales consumed
                 }
-                if (i >= 1) rescale(i - 1, pend_scale, pend_end, pend_whole, pend_first, pend_tile);
                 // this group ends a segment at the tile's last group or the range's last
-                const bool last_of_chunk = gq == GPC - 1;
-                const bool seg_end = last_of_chunk && (cur_chunk == nchunks - 1 || c == nit - 1);
-                pend_scale = sc;
-                pend_end = seg_end;
-                pend_whole = seg_end && (c - seg_start) == cur_chunk && cur_chunk == nchunks - 1;
-                pend_first = seg_start == 0;
-                pend_tile = cur_tile;
+                const bool seg_end = gq == GPC - 1 && (cur_chunk == nchunks - 1 || c == nit - 1);
+                const Pend cur{sc, seg_end,
+                               seg_end && (c - seg_start) == cur_chunk && cur_chunk == nchunks - 1,
+                               seg_start == 0, cur_tile};
                 if (seg_end) seg_start = c + 1;
+                if constexpr (LAG == 2) {
+                    if (i >= 2) rescale(i - 2, p0);
+                    p0 = p1;
+                    p1 = cur;
+                } else {
+                    if (i >= 1) rescale(i - 1, p0);
+                    p0 = cur;
+                }
             }
             if (++cur_chunk == nchunks) {
                 cur_chunk = 0;
@@ -425,7 +460,12 @@ __global__ void __launch_bounds__(kTcThreads, TcCfg<NT>::ctas_per_sm)
                 ph ^= 1u;
             }
         }
-        if (i >= 1) rescale(i - 1, pend_scale, pend_end, pend_whole, pend_first, pend_tile);
+        if constexpr (LAG == 2) {
+            if (i >= 2) rescale(i - 2, p0);
+            if (i >= 1) rescale(i - 1, p1);
+        } else {
+            if (i >= 1) rescale(i - 1, p0);
+        }
     }
 
     tc_fence_before();
