@@ -129,10 +129,12 @@ class ClockSampler:
 
 # --------------------------------------------------------------- workload
 def build_llama3_8b(q4, wl, torch, layers, rank, B, device):
-    """Quantized weights of `layers` distinct Llama-3-8B layers (sym g128)."""
+    """Quantized weights of `layers` distinct Llama-3-8B layers (sym g128);
+    each rank's replica draws its own layers."""
+    from post_weight_quantization_group_b200.replicas import replica_layer
     mats = []
     for layer in range(layers):
-        seeds = wl.llama3_8b_layer_seeds(layer + 1000 * rank)
+        seeds = wl.llama3_8b_layer_seeds(replica_layer(layer, rank))
         for name, (out, inn) in wl.LLAMA3_8B.items():
             W = wl.normal_weight(out, inn, seeds[name], device=device)
             mats.append((name, q4.q4_quantize_pack(W, 128, True)))
@@ -223,6 +225,7 @@ def run_ours(args):
 
     import post_weight_quantization_group_b200 as q4
     from post_weight_quantization_group_b200 import workloads as wl
+    from post_weight_quantization_group_b200.replicas import aggregate_throughput, max_over_ranks
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -270,12 +273,9 @@ def run_ours(args):
     ms_eager = time_region(torch, step, max(3, args.steps // 10), 2, stream)
     ms_eager /= max(3, args.steps // 10)
 
-    t = torch.tensor([ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dist, device)
     ms_per_step = ms_max / args.steps
-    value = world * step_bytes * args.steps / (ms_max * 1e-3) / 1e9
+    value = aggregate_throughput(step_bytes * args.steps, ms_max * 1e-3, world) / 1e9
 
     # ---- bf16 reference on one layer of the same shapes (436 MB > L2)
     bf_mats = []
@@ -335,10 +335,8 @@ def run_ours(args):
     t0 = time.perf_counter()
     for _ in range(ne):
         e2e_step()
-    e2e_s = torch.tensor([time.perf_counter() - t0], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(e2e_s, op=dist.ReduceOp.MAX)
-    e2e_value = world * step_bytes * ne / float(e2e_s.item()) / 1e9
+    e2e_s = max_over_ranks(time.perf_counter() - t0, dist, device)
+    e2e_value = aggregate_throughput(step_bytes * ne, e2e_s, world) / 1e9
 
     clocks = clk.summary()
     peak = peaks["hbm_gbs"]
