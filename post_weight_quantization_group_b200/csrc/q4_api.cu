@@ -250,7 +250,7 @@ constexpr int kGemvRT = kGemvCW * kGemvMT * 16;
 constexpr int kSkCW = Q4_SK_CW;
 constexpr int kSkRT = kSkCW * 16;
 constexpr int kSkCtasPerSm = 2;
-constexpr int kSkMinIters = 4;
+constexpr int kSkMinIters = 2;
 
 // Workspace layout, the same for every shape, batch and kernel so that one
 // buffer can serve any sequence of calls: [one counter per row tile, at most

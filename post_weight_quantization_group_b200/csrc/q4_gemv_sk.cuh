@@ -327,7 +327,10 @@ __global__ void __launch_bounds__((CW + 2) * 32, 2)
 
     bool ok = true;
     for (int c = 0; c < nit; ++c) {
-        if (ok) ok = mbar_wait_bounded(&full[s], ph, status, kWaitLimitNs);
+        // One wait per stage: the helper arrives on sxful only after it has
+        // observed the TMA loads of the stage complete (full), so by the
+        // release/acquire chain the weights and scales are visible here too;
+        // each mbarrier wait costs ~100 cycles even when the phase is done.
         if (ok) ok = mbar_wait_bounded(&sxful[s], ph, status, kWaitLimitNs);
         if (ok) {
             const uint32_t sa = sbase + sbytes * static_cast<uint32_t>(s);
