@@ -32,7 +32,7 @@
  *  - the decode product y = x W^T of the dequantised weights:
  *    arganzheng.life section 二.1 ([B,k] x [k,n] decode GEMM) and 二.3.
  *
- * Readings taken where the pages leave a step open (all listed in the design doc):
+ * Readings taken where the pages leave a step open:
  *  - the scale is computed in fp32 (IEEE division), stored as fp16, and the
  *    STORED fp16 scale is the one that quantizes and dequantizes;
  *  - round() is round-half-to-even (torch.round in the ybb.press code);
