@@ -42,7 +42,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # gate_proj launch whose algorithmic bytes are 30.28 MB).  Scaled to the
 # bench's average launch; it must be re-taken whenever the kernel changes.
 GEMV_TRAFFIC_RATIO = 30.33 / 30.28
-GEMV_TRAFFIC_SOURCE = ("ncu --set full on one 14336x4096 B=1 launch "
+GEMV_TRAFFIC_SOURCE = ("ncu --set full on one 14336x4096 B=1 launch of the current kernel "
                        "(profiles/q4_gemv_sk_llama3_8b_gate_full.txt), scaled by algorithmic bytes")
 
 
