@@ -306,7 +306,9 @@ q4_status run_gemv(const q4_weight* w, const void* x, int64_t B, void* y, int yd
     const SkPlan p = sk_plan(w->out, w->in, sm_count(dev));
     if (!ws || ws_bytes < p.ws_bytes) return Q4_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return Q4_ERR_ALIGNMENT;
-    // deepest ring that still lets two CTAs share an SM
+    // Deepest ring that still lets two CTAs share an SM.  From B = 4 on, two
+    // helper warps split the activation work; they need an even ring (each
+    // owns fixed slots), so the ring is cut to an even depth.
     const int per_sm = 228 * 1024;
     int stages = kSkMaxStages;
     SkGeom geo = sk_geom(kSkRT, stages, static_cast<int>(B), SYM);
@@ -314,6 +316,9 @@ q4_status run_gemv(const q4_weight* w, const void* x, int64_t B, void* y, int yd
         --stages;
         geo = sk_geom(kSkRT, stages, static_cast<int>(B), SYM);
     }
+    const bool two_helpers = B >= 4;
+    if (two_helpers && (stages & 1)) geo = sk_geom(kSkRT, --stages, static_cast<int>(B), SYM);
+    const int helpers = two_helpers ? 2 : 1;
     const int64_t G = w->in / GS;
     // scale / zero windows by TMA when their rows are 16-byte aligned
     const bool meta_tma = (G % 8) == 0 && aligned(w->scales, 16) && (SYM || aligned(w->zeros, 16));
@@ -339,14 +344,15 @@ q4_status run_gemv(const q4_weight* w, const void* x, int64_t B, void* y, int yd
                                   8, CU_TENSOR_MAP_SWIZZLE_NONE))
             return Q4_ERR_CUDA;
     }
-    auto kernel = q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW>;
+    auto kernel = two_helpers ? q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 2>
+                              : q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 1>;
     if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), false)) return Q4_ERR_CUDA;
     unsigned* status = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
         return Q4_ERR_CUDA;
     unsigned* ws_count = reinterpret_cast<unsigned*>(ws);
     float* ws_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kWsCounterBytes);
-    return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3((kSkCW + 2) * 32),
+    return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3((kSkCW + 1 + helpers) * 32),
                           geo.total, 1, true, st, tmap_w, tmap_x, tmap_s, tmap_z, meta_tma ? 1 : 0,
                           reinterpret_cast<const uint16_t*>(w->scales),
                           reinterpret_cast<const uint16_t*>(w->zeros), stages,

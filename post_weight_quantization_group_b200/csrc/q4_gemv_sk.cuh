@@ -26,9 +26,10 @@
 //    [B rows x 256 values] and the aligned window of 8 groups of scales
 //    (and zero points) [RT rows x 8] that holds the chunk's groups, into a
 //    ring of `stages` shared-memory stages;
-//  * a helper warp: per stage it rewrites the activation chunk in MMA
-//    fragment order and sums it per group, shared memory to shared memory,
-//    so the consumer threads do nothing but unpack, multiply and rescale.
+//  * one helper warp (two for B >= 4, taking alternate chunks): per stage it
+//    rewrites the activation chunk in MMA fragment order and sums it per
+//    group, shared memory to shared memory, so the consumer threads do
+//    nothing but unpack, multiply and rescale.
 //    (Scale rows that are not 16-byte aligned cannot be copied by TMA; the
 //    helper then loads the chunk's scales itself.)
 //
@@ -56,23 +57,28 @@ namespace q4dev {
 constexpr int kSkMaxStages = 4;
 
 struct SkGeom {
-    size_t off_x, off_xp, off_sx, off_sc, off_zc, stage_bytes, off_bar, total;
+    size_t w_bytes, off_m, m_bytes;              // weight tiles, per-stage slots
+    size_t off_x, off_xp, off_sx, off_sc, off_zc;  // inside a per-stage slot
+    size_t off_bar, total;
 };
 
-// Per stage: weights [rt x 128 B] | activations as loaded [b x 512 B] |
-// activations in fragment order [8 slots x 8 batch x 4 threads x 16 B] |
-// group sums [8 groups x 8 batch] fp32 | scale window [rt x 8] fp16 |
-// zero-point window [rt x 8] fp16 (asymmetric only).
+// All stages' weight tiles [rt x 128 B] first (each 1024-byte aligned for
+// the 128-byte swizzle), then per stage: activations [b x 512 B] as loaded,
+// rewritten in place by the helper into MMA fragment order [8 slots x 8
+// batch x 4 threads x 16 B] | group sums [8 groups x 8 batch] fp32 | scale
+// window [rt x 8] fp16 | zero-point window [rt x 8] fp16 (asymmetric only).
 __host__ __device__ inline SkGeom sk_geom(int rt, int stages, int b, bool sym) {
     SkGeom g{};
-    g.off_x = static_cast<size_t>(rt) * kChunkBytes;
-    g.off_xp = g.off_x + align_up(static_cast<size_t>(b) * 512, 128);
-    g.off_sx = g.off_xp + 8 * 8 * 64;
+    (void)b;  // the activation area is 8 x 512 B for every b <= 8
+    g.w_bytes = static_cast<size_t>(rt) * kChunkBytes;
+    g.off_m = g.w_bytes * stages;
+    g.off_x = 0;
+    g.off_xp = 0;
+    g.off_sx = 8 * 8 * 64;
     g.off_sc = g.off_sx + 8 * 8 * 4;
     g.off_zc = g.off_sc + static_cast<size_t>(rt) * 16;
-    const size_t end = g.off_zc + (sym ? 0 : static_cast<size_t>(rt) * 16);
-    g.stage_bytes = align_up(end, 1024);
-    g.off_bar = g.stage_bytes * stages;
+    g.m_bytes = align_up(g.off_zc + (sym ? 0 : static_cast<size_t>(rt) * 16), 128);
+    g.off_bar = align_up(g.off_m + g.m_bytes * stages, 8);
     g.total = g.off_bar + static_cast<size_t>(3 * kSkMaxStages) * 8 + 64 + 1024;
     return g;
 }
@@ -94,8 +100,12 @@ __device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v
     return old;
 }
 
-template <bool BF16, int GS, bool SYM, int CW>
-__global__ void __launch_bounds__((CW + 2) * 32, 2)
+// NH helper warps per CTA: the helper's per-chunk work grows with B, so
+// larger batches split the chunks between two helpers (chunk c to helper
+// c % 2).  NH is a template parameter so that each variant gets the register
+// budget of its own block size.
+template <bool BF16, int GS, bool SYM, int CW, int NH>
+__global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
     q4_gemv_sk_kernel(const __grid_constant__ CUtensorMap tmap_w,
                       const __grid_constant__ CUtensorMap tmap_x,
                       const __grid_constant__ CUtensorMap tmap_s,
@@ -137,17 +147,8 @@ __global__ void __launch_bounds__((CW + 2) * 32, 2)
         }
         fence_mbarrier_init_cluster();
     }
-    // activation rows n >= B of every stage stay zero: the consumers load
-    // all 8 rows without a branch
-    for (int i = threadIdx.x; i < stages * 8 * 8 * 4; i += blockDim.x) {
-        const int s = i / (8 * 8 * 4);
-        const int slot = (i / 32) % 8;
-        const int n = (i / 4) % 8;
-        const int t = i % 4;
-        if (n >= B)
-            *reinterpret_cast<uint4*>(smem + geo.stage_bytes * s + geo.off_xp +
-                                      ((slot * 8 + n) * 4 + t) * 16) = make_uint4(0, 0, 0, 0);
-    }
+    // fragment-order rows n >= B are never read: consumer threads of batch
+    // columns n >= B skip their activation loads
     __syncthreads();
     grid_launch_dependents();
 
@@ -163,13 +164,13 @@ __global__ void __launch_bounds__((CW + 2) * 32, 2)
             {
                 int tile = tile0, chunk = chunk0;
                 for (int c = 0; c < pre; ++c) {
-                    uint8_t* st = smem + geo.stage_bytes * c;
+                    uint8_t* ms = smem + geo.off_m + geo.m_bytes * c;
                     mbar_arrive_expect_tx(&full[c], tx);
-                    tma_load_2d(st, &tmap_w, chunk * kChunkBytes, tile * RT, &full[c]);
+                    tma_load_2d(smem + geo.w_bytes * c, &tmap_w, chunk * kChunkBytes, tile * RT, &full[c]);
                     if (meta_tma) {
                         const int win = (chunk * GPC) & ~7;
-                        tma_load_2d(st + geo.off_sc, &tmap_s, win, tile * RT, &full[c]);
-                        if constexpr (!SYM) tma_load_2d(st + geo.off_zc, &tmap_z, win, tile * RT, &full[c]);
+                        tma_load_2d(ms + geo.off_sc, &tmap_s, win, tile * RT, &full[c]);
+                        if constexpr (!SYM) tma_load_2d(ms + geo.off_zc, &tmap_z, win, tile * RT, &full[c]);
                     }
                     if (++chunk == nchunks) {
                         chunk = 0;
@@ -184,17 +185,17 @@ __global__ void __launch_bounds__((CW + 2) * 32, 2)
             for (int c = 0; c < nit && ok; ++c) {
                 if (c >= stages) ok = mbar_wait_bounded(&empty[s], ph ^ 1u, status, kWaitLimitNs);
                 if (!ok) break;
-                uint8_t* st = smem + geo.stage_bytes * s;
+                uint8_t* ms = smem + geo.off_m + geo.m_bytes * s;
                 if (c >= pre) {
                     mbar_arrive_expect_tx(&full[s], tx);
-                    tma_load_2d(st, &tmap_w, chunk * kChunkBytes, tile * RT, &full[s]);
+                    tma_load_2d(smem + geo.w_bytes * s, &tmap_w, chunk * kChunkBytes, tile * RT, &full[s]);
                     if (meta_tma) {
                         const int win = (chunk * GPC) & ~7;
-                        tma_load_2d(st + geo.off_sc, &tmap_s, win, tile * RT, &full[s]);
-                        if constexpr (!SYM) tma_load_2d(st + geo.off_zc, &tmap_z, win, tile * RT, &full[s]);
+                        tma_load_2d(ms + geo.off_sc, &tmap_s, win, tile * RT, &full[s]);
+                        if constexpr (!SYM) tma_load_2d(ms + geo.off_zc, &tmap_z, win, tile * RT, &full[s]);
                     }
                 }
-                tma_load_2d(st + geo.off_x, &tmap_x, chunk * kChunkCodes, 0, &full[s]);
+                tma_load_2d(ms + geo.off_x, &tmap_x, chunk * kChunkCodes, 0, &full[s]);
                 if (++chunk == nchunks) {
                     chunk = 0;
                     ++tile;
@@ -213,8 +214,10 @@ __global__ void __launch_bounds__((CW + 2) * 32, 2)
         return;
     }
 
-    if (warp == CW + 1) {
-        // --------------------------------------------------------- helper
+    if (warp >= CW + 1) {
+        // -------------------------------------------------------- helpers
+        // helper hw of nh (launched warps beyond the producer) takes the
+        // chunks c with c % nh == hw
         // Lane l owns the 8-value block l of each activation row of a chunk
         // (256 = 32 x 8): it stores the block pair-permuted at the fragment
         // slot of the consumer thread that multiplies those codes, and adds
@@ -224,20 +227,46 @@ __global__ void __launch_bounds__((CW + 2) * 32, 2)
         const int rem = lane % (GS / 8);
         const int ht = rem / WPG;
         const int hi = rem % WPG;
+        // A helper must own fixed ring slots: waiting for phase k of a slot
+        // before phase k-1 is known complete would read the parity of phase
+        // k-1 as done.  So nh divides the ring depth; otherwise one helper.
+        const int hw = warp - (CW + 1);
+        const int nh = stages % NH == 0 ? NH : 1;
+        if (hw >= nh) return;
         grid_dependency_wait();
         int tile = tile0, chunk = chunk0, s = 0;
         uint32_t ph = 0;
-        const uint32_t sbase = smem_u32(smem);
-        const uint32_t sbytes = static_cast<uint32_t>(geo.stage_bytes);
+        const uint32_t sbase = smem_u32(smem) + static_cast<uint32_t>(geo.off_m);
+        const uint32_t sbytes = static_cast<uint32_t>(geo.m_bytes);
         const uint32_t oX = static_cast<uint32_t>(geo.off_x), oXP = static_cast<uint32_t>(geo.off_xp);
         const uint32_t oSX = static_cast<uint32_t>(geo.off_sx);
         const uint32_t xp_lane = oXP + static_cast<uint32_t>((((hgq * WPG + hi) * 8) * 4 + ht) * 16);
         for (int c = 0; c < nit; ++c) {
+            if (c % nh != hw) {  // another helper's chunk
+                if (++chunk == nchunks) {
+                    chunk = 0;
+                    ++tile;
+                }
+                if (++s == stages) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+                continue;
+            }
             if (!mbar_wait_bounded(&full[s], ph, status, kWaitLimitNs)) break;
-            uint8_t* st = smem + geo.stage_bytes * s;
+            uint8_t* st = smem + geo.off_m + geo.m_bytes * s;
             const uint32_t sa = sbase + sbytes * static_cast<uint32_t>(s);
-            for (int n = 0; n < B; ++n) {
-                const uint4 q = lds128(sa + oX + n * 512 + lane * 16);
+            // the fragment order overwrites the activations in place: every
+            // lane reads its blocks of all rows before any lane writes
+            uint4 qv[8];
+#pragma unroll
+            for (int n = 0; n < 8; ++n)
+                if (n < B) qv[n] = lds128(sa + oX + n * 512 + lane * 16);
+            __syncwarp();
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                if (n >= B) break;
+                const uint4 q = qv[n];
                 uint4 o;
                 o.x = pair_lo(q.x, q.z);  // (x0, x4)
                 o.y = pair_hi(q.x, q.z);  // (x1, x5)
@@ -315,8 +344,10 @@ __global__ void __launch_bounds__((CW + 2) * 32, 2)
     grid_dependency_wait();  // y and the workspace are written below
 
     // 32-bit shared addresses of this thread's loads inside a stage
-    const uint32_t sbase = smem_u32(smem);
-    const uint32_t sbytes = static_cast<uint32_t>(geo.stage_bytes);
+    const uint32_t wbase = smem_u32(smem);
+    const uint32_t wbytes = static_cast<uint32_t>(geo.w_bytes);
+    const uint32_t sbase = wbase + static_cast<uint32_t>(geo.off_m);
+    const uint32_t sbytes = static_cast<uint32_t>(geo.m_bytes);
     const uint32_t a_xp = static_cast<uint32_t>(geo.off_xp) + (gid * 4 + t) * 16;
     const uint32_t a_sx = static_cast<uint32_t>(geo.off_sx) + 2 * t * 4;
     const uint32_t a_sc0 = static_cast<uint32_t>(geo.off_sc) + R0 * 16;
@@ -347,7 +378,7 @@ __global__ void __launch_bounds__((CW + 2) * 32, 2)
                     xf[i][3] = v.w;
                 }
                 uint32_t w0[WPG], w1[WPG];
-                const uint32_t p0 = sa + a_w[gq];
+                const uint32_t p0 = wbase + wbytes * static_cast<uint32_t>(s) + a_w[gq];
                 const uint32_t p1 = p0 + 8 * kChunkBytes;
                 if constexpr (WPG == 4) {
                     const uint4 a = lds128(p0);
