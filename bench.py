@@ -39,7 +39,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic of q4_gemv_sk_kernel per algorithmic byte, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum = 30.33 MB on a 14336 x 4096
-# gate_proj launch whose algorithmic bytes are 30.28 MB).  Scaled to the
+# gate_proj launch whose algorithmic bytes are 30.28 MB; same ratio in every
+# capture of this kernel so far).  Scaled to the
 # bench's average launch; it must be re-taken whenever the kernel changes.
 GEMV_TRAFFIC_RATIO = 30.33 / 30.28
 GEMV_TRAFFIC_SOURCE = ("ncu --set full on one 14336x4096 B=1 launch of the current kernel "
@@ -366,7 +367,7 @@ def run_ours(args):
                      "traffic": round(step_bytes / launches_per_step * GEMV_TRAFFIC_RATIO),
                      "traffic_unit": "DRAM bytes per launch",
                      "traffic_source": GEMV_TRAFFIC_SOURCE,
-                     "kernel": "q4_gemv_sk_kernel<bf16,g128,sym,8>",
+                     "kernel": "q4_gemv_sk_kernel<bf16,g128,sym,8,1>",
                      "bytes_per_launch_avg": step_bytes // launches_per_step},
         "clocks": clocks,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
