@@ -211,12 +211,14 @@ Q4_API q4_status q4_gemv_noalloc(const q4_weight* w, const void* x, q4_dtype x_d
                                  void* y, q4_dtype y_dtype, q4_stream stream);
 
 /*
- * The unquantised bf16 product y = x W^T with fp32 accumulation, the
+ * The unquantised bf16 product y = x W^T with fp32 accumulation, a
  * baseline the INT4 path is compared against and the probe of the bandwidth
  * a weight stream reaches (ybb.press section 一, roofline_bound; arganzheng.
  * life section 二.4, BF16 vs W4A16 batch table).
- *   W [out, in] bf16, x [B, in] bf16, y [B, out] bf16; 1 <= B <= 128;
- *   `in` a multiple of 64; W, x, y 16-byte aligned.
+ *   W [out, in] bf16, x [B, in] bf16, y [B, out] bf16; `in` a multiple of 64;
+ *   W, x, y 16-byte aligned.
+ *   1 <= B <= 8 runs here; 9 <= B <= 128 returns Q4_ERR_UNSUPPORTED (a plain
+ *   library GEMM is the bf16 baseline there); other B Q4_ERR_SHAPE.
  */
 Q4_API q4_status bf16_gemv_ref_bw(const void* W, int64_t out, int64_t in, const void* x, int64_t B,
                            void* y, q4_stream stream);

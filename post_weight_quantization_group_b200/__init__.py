@@ -257,7 +257,8 @@ def q4_gemv_noalloc(w: Q4Weight, x: torch.Tensor, y: torch.Tensor | None = None,
 
 def bf16_gemv_ref_bw(W: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None,
                      stream=None) -> torch.Tensor:
-    """y = x W^T for bf16 W [out, in], x [B, in], B <= 128."""
+    """y = x W^T for bf16 W [out, in], x [B, in], B <= 8 (larger B:
+    Q4_ERR_UNSUPPORTED)."""
     lib = load_library()
     out, inn = W.shape
     B = x.shape[0]

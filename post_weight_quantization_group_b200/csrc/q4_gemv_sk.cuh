@@ -335,7 +335,6 @@ __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
         swo[gq] = (((byte >> 4) ^ (R0 & 7)) << 4) | (byte & 15);
     }
     // batch columns n >= B are zero: their threads skip the activation loads
-    // (shared-memory bandwidth, not arithmetic, bounds this loop)
     const bool x_live = gid < B;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     int seg_start = 0;  // first iteration (relative) of the current segment
