@@ -78,6 +78,10 @@ def _load():
     lib.oracle_gemv_f64.restype = ctypes.c_int
     lib.oracle_dense_rows_f64.argtypes = [P, I64, I64, P, I64, P, I64, P]
     lib.oracle_dense_rows_f64.restype = ctypes.c_int
+    lib.oracle_clip_search_group.argtypes = [P, I32, I32, P, P]
+    lib.oracle_clip_search_group.restype = I32
+    lib.oracle_quantize_pack_clip.argtypes = [P, I64, I64, I32, I32, P, P, P]
+    lib.oracle_quantize_pack_clip.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -155,6 +159,32 @@ def quantize_pack(W: np.ndarray, group_size: int, symmetric: bool):
     if rc != 0:
         raise ValueError("oracle_quantize_pack rejected its arguments")
     return q, s, z
+
+
+def quantize_pack_clip(W: np.ndarray, group_size: int, n_alpha: int):
+    """Symmetric INT4 with the per-group range search (see
+    oracle_clip_search_group).  Returns (qweight uint8 [out, in/2], scales
+    uint16 fp16-bits [out, in/g], alpha index int32 [out, in/g])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    out, inn = W.shape
+    G = inn // group_size
+    q = np.zeros((out, inn // 2), dtype=np.uint8)
+    s = np.zeros((out, G), dtype=np.uint16)
+    idx = np.zeros((out, G), dtype=np.int32)
+    rc = _load().oracle_quantize_pack_clip(_ptr(W), out, inn, int(group_size), int(n_alpha),
+                                           _ptr(q), _ptr(s), _ptr(idx))
+    if rc != 0:
+        raise ValueError("oracle_quantize_pack_clip rejected its arguments")
+    return q, s, idx
+
+
+def clip_errors(w: np.ndarray, n_alpha: int):
+    """One group: (chosen index, fp64 errors E_j [n], fp16 scale bits [n])."""
+    w = np.ascontiguousarray(w, dtype=np.float32).ravel()
+    err = np.zeros(n_alpha, dtype=np.float64)
+    s16 = np.zeros(n_alpha, dtype=np.uint16)
+    best = _load().oracle_clip_search_group(_ptr(w), int(w.size), int(n_alpha), _ptr(err), _ptr(s16))
+    return int(best), err, s16
 
 
 def code_at(qweight: np.ndarray, inn: int, r: int, k: int, symmetric: bool) -> int:

@@ -229,6 +229,86 @@ ORACLE_API int oracle_quantize_pack(const float* W, int64_t out, int64_t in, int
     return 0;
 }
 
+/*
+ * Range (clipping) search of symmetric INT4 group quantization
+ * ("post-training-quantization-gptq-awq-and-rotation" (arganzheng.life),
+ * section 三.2, 裁剪与舍入的权衡: scan a set of ranges alpha between 0.8 and
+ * 1.0 of max|w| and keep the one with the smallest error).  Readings:
+ *  - candidates alpha_j = amax (K - j) / K, j = 0 .. n-1, K = 5 (n - 1)
+ *    (alpha_0 = amax, alpha_{n-1} = 0.8 amax; n = 1: amax only);
+ *  - s_j = fp16(fp32(amax (K - j)) / fp32(7 K)) with IEEE division; the
+ *    product and 7 K are exact in fp32, so s_0 is bit-for-bit the RTN scale;
+ *  - codes q = clamp(rne(w / s_j), -7, 7): the section's symmetric grid of
+ *    2^b - 1 points (RTN's -8 is unreachable at alpha = amax, so j = 0
+ *    reproduces RTN's codes);
+ *  - error E_j = sum over the group of (w - s_j q)^2 in fp64; a candidate
+ *    whose fp16 scale is 0 is skipped unless it is the first;
+ *  - j replaces the best so far only if E_j < E_best (1 - 1e-12), so ties
+ *    keep the wider range.
+ * Fills the group's E_j (and fp16 scale bits) for j < n; returns the index.
+ */
+ORACLE_API int32_t oracle_clip_search_group(const float* w, int32_t g, int32_t n,
+                                            double* err, uint16_t* s16_out) {
+    float a = 0.0f;
+    for (int32_t k = 0; k < g; ++k) {
+        float m = fabsf(w[k]);
+        if (m > a) a = m;
+    }
+    const int32_t K = 5 * (n - 1);
+    int32_t best = 0;
+    double best_e = 0.0;
+    for (int32_t j = 0; j < n; ++j) {
+        const float num = (n == 1) ? a : a * (float)(K - j);
+        const float den = (n == 1) ? 7.0f : 7.0f * (float)K;
+        const uint16_t s16 = oracle_f32_to_f16(num / den);
+        const float sf = oracle_f16_to_f32(s16);
+        double e = 0.0;
+        for (int32_t k = 0; k < g; ++k) {
+            const int32_t q = (sf == 0.0f) ? 0 : oracle_quantize_value(w[k], sf, 0, -7, 7);
+            const double d = (double)w[k] - (double)sf * (double)q;
+            e += d * d;
+        }
+        if (err) err[j] = e;
+        if (s16_out) s16_out[j] = s16;
+        if (j == 0) {
+            best_e = e;
+        } else if (sf != 0.0f && e < best_e * (1.0 - 1e-12)) {
+            best = j;
+            best_e = e;
+        }
+    }
+    return best;
+}
+
+/* Symmetric INT4 quantization with the range search above, packed like
+ * oracle_quantize_pack; alpha_idx (may be NULL) receives each group's j. */
+ORACLE_API int oracle_quantize_pack_clip(const float* W, int64_t out, int64_t in, int32_t g,
+                                         int32_t n, uint8_t* qweight, uint16_t* scales,
+                                         int32_t* alpha_idx) {
+    if (g <= 0 || in <= 0 || out < 0 || (in % g) != 0 || (g % 2) != 0 || n < 1 || n > 64)
+        return -1;
+    const int64_t G = in / g;
+    uint16_t* s16 = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)n);
+    if (!s16) return -1;
+    for (int64_t r = 0; r < out; ++r) {
+        for (int64_t j = 0; j < G; ++j) {
+            const float* w = W + r * in + j * g;
+            const int32_t best = oracle_clip_search_group(w, g, n, NULL, s16);
+            const float sf = oracle_f16_to_f32(s16[best]);
+            scales[r * G + j] = s16[best];
+            if (alpha_idx) alpha_idx[r * G + j] = best;
+            uint8_t* dst = qweight + r * (in / 2) + j * (g / 2);
+            for (int32_t k = 0; k < g; k += 2) {
+                const int32_t q0 = (sf == 0.0f) ? 0 : oracle_quantize_value(w[k], sf, 0, -7, 7);
+                const int32_t q1 = (sf == 0.0f) ? 0 : oracle_quantize_value(w[k + 1], sf, 0, -7, 7);
+                dst[k / 2] = (uint8_t)((q0 & 0xF) | ((q1 & 0xF) << 4));
+            }
+        }
+    }
+    free(s16);
+    return 0;
+}
+
 /* Unpack one code: low nibble for even k, high for odd k; symmetric codes are
  * two's complement 4-bit integers, asymmetric codes are unsigned. */
 ORACLE_API int32_t oracle_code_at(const uint8_t* qweight, int64_t in, int64_t r, int64_t k,

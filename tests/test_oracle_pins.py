@@ -367,3 +367,78 @@ def test_bits_per_weight_accounting():
         assert abs(bits_codes_scales + 4 / gs - row["bits_per_weight"]) < 1e-3 + 1e-9
         assert abs((q.nbytes + s.nbytes + z.nbytes) * 8 / n - (4 + 32 / gs)) < 1e-12
     assert abs((4 + 32 / 128) - g["fp16_scale_fp16_zero_g128"]) < 1e-12
+
+
+# ---------------------------------------------- range (clipping) search
+# arganzheng.life post-training-quantization-gptq-awq-and-rotation, section
+# 三.2: scan ranges alpha from 0.8 to 1.0 of max|w|, keep the smallest error.
+
+def _clip_reference(w, n):
+    """Independent numpy restatement of one group's search: candidate fp16
+    scales, codes rint(w / s) clamped to +-7, fp64 squared error, ties to
+    the wider range."""
+    w = np.asarray(w, dtype=np.float32)
+    a = np.float32(np.max(np.abs(w)))
+    K = 5 * (n - 1)
+    errs, scales = [], []
+    for j in range(n):
+        num = a if n == 1 else np.float32(a * np.float32(K - j))
+        den = np.float32(7.0) if n == 1 else np.float32(7 * K)
+        s = np.float32(np.float16(np.float32(num) / den))
+        q = np.zeros_like(w) if s == 0 else np.clip(np.rint(w / s), -7, 7)
+        d = w.astype(np.float64) - np.float64(s) * q.astype(np.float64)
+        errs.append(float(np.sum(d * d)))
+        scales.append(s)
+    best = 0
+    for j in range(1, n):
+        if scales[j] != 0 and errs[j] < errs[best] * (1 - 1e-12):
+            best = j
+    return best, np.array(errs), np.array(scales)
+
+
+def test_clip_search_single_candidate_is_rtn():
+    W = wl.normal_weight(48, 1024, 41).float().numpy()
+    q1, s1, idx = oracle.quantize_pack_clip(W, 128, 1)
+    qr, sr, _ = oracle.quantize_pack(W, 128, True)
+    assert np.array_equal(q1, qr) and np.array_equal(s1, sr) and not idx.any()
+
+
+@pytest.mark.parametrize("kind", ["normal", "t3", "uniform"])
+def test_clip_search_matches_independent_restatement(kind):
+    gen = {"normal": wl.normal_weight, "t3": wl.student_t_weight, "uniform": wl.uniform_weight}[kind]
+    W = gen(16, 512, 42).float().numpy()
+    for r in range(16):
+        for j in range(4):
+            w = W[r, j * 128:(j + 1) * 128]
+            best, err, s16 = oracle.clip_errors(w, 21)
+            rbest, rerr, rs = _clip_reference(w, 21)
+            assert best == rbest
+            assert np.allclose(err, rerr, rtol=1e-12, atol=0)
+            assert np.array_equal(s16.view(np.float16).astype(np.float32), rs)
+
+
+def test_clip_search_never_worse_than_rtn_and_grid_refinement():
+    W = wl.student_t_weight(64, 1024, 43).float().numpy()
+    for n_small, n_big in [(21, 41), (5, 9)]:
+        _, _, _ = oracle.quantize_pack_clip(W, 128, n_small)
+        for r in range(0, 64, 7):
+            for j in range(8):
+                w = W[r, j * 128:(j + 1) * 128]
+                b1, e1, _ = oracle.clip_errors(w, 1)
+                bs, es, _ = oracle.clip_errors(w, n_small)
+                bb, eb, _ = oracle.clip_errors(w, n_big)
+                assert es[bs] <= e1[0]                      # candidate 0 is RTN
+                assert eb[bb] <= es[bs] * (1 + 1e-12)        # the small grid is a subset
+
+
+def test_clip_search_gaussian_optimum_below_max():
+    """For large Gaussian groups the best range lies well below max|w| (the
+    section puts the 4-bit optimum at 2.5-3 sigma against a max of 4-5
+    sigma): every group of 4096 picks the grid's floor, 0.8 max."""
+    W = wl.normal_weight(32, 4096, 44).float().numpy()
+    _, _, idx = oracle.quantize_pack_clip(W, 4096, 21)
+    assert np.all(idx == 20)
+    sigma = 0.02
+    amax = np.abs(W).max(axis=1) / sigma
+    # the floor 0.8 max lies at or above 2.5 sigma: the optimum is below it
+    assert np.all(0.8 * amax > 2.5) and np.median(amax) > 3.5
