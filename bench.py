@@ -321,7 +321,18 @@ def run_ours(args):
 
     nq = max(10, args.steps // 20)
     ms_q = time_region(torch, q_step, nq, 2, stream) / nq
-    del qW, qouts
+
+    # ---- the same with the per-group range (clipping) search over 21 ranges
+    def qc_step():
+        for (n, W), (qo, so) in zip(qW, qouts):
+            q4.q4_quantize_pack_clip(W, 128, 21, qweight=qo, scales=so)
+
+    nqc = max(3, args.steps // 200)
+    ms_qc = time_region(torch, qc_step, nqc, 1, stream) / nqc
+    Wg = dict(qW)["gate_proj"]
+    mse_clip = (q4.q4_dequant(q4.q4_quantize_pack_clip(Wg, 128, 21)) - Wg.float()).pow(2).mean().item()
+    mse_rtn = (q4.q4_dequant(q4.q4_quantize_pack(Wg, 128, True)) - Wg.float()).pow(2).mean().item()
+    del qW, qouts, Wg
 
     # ---- end to end through the public API with host buffers
     x_host = {k: v.cpu().pin_memory() for k, v in xs.items()}
@@ -374,6 +385,9 @@ def run_ours(args):
                  "cublas_us_per_layer": round(ms_cublas * 1e3, 3)},
         "quantize_pack": {"gbs": round(qbytes / (ms_q * 1e-3) / 1e9, 1),
                           "us_per_layer": round(ms_q * 1e3, 2)},
+        "quantize_pack_clip": {"n_alpha": 21, "gbs": round(qbytes / (ms_qc * 1e-3) / 1e9, 1),
+                               "us_per_layer": round(ms_qc * 1e3, 2),
+                               "weight_mse_vs_rtn": round(mse_clip / mse_rtn, 4)},
         "roofline": {"bound": "hbm", "achieved": round(value / world, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(value / world / peak, 4),
                      "peak_kind": peak_kind,

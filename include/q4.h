@@ -112,6 +112,30 @@ Q4_API q4_status q4_quantize_pack(const void* W, q4_dtype w_dtype, int64_t out, 
                            uint8_t* qweight, void* scales, void* zeros, q4_stream stream);
 
 /*
+ * Symmetric group-wise INT4 quantization with a per-group range (clipping)
+ * search ("post-training-quantization-gptq-awq-and-rotation" (arganzheng.life)
+ * section 三.2, 裁剪与舍入的权衡: scan ranges alpha from 0.8 to 1.0 of max|w|
+ * and keep the one with the smallest error).  Candidates
+ *   alpha_j = amax (K - j) / K,   j = 0 .. n_alpha-1,   K = 5 (n_alpha - 1),
+ *   s_j = fp16(amax (K - j) / (7 K))   (IEEE fp32 division),
+ *   q = clamp(rne(w / s_j), -7, 7)     (the section's symmetric grid),
+ *   E_j = sum over the group of (w - s_j q)^2 in fp64;
+ * candidate j replaces the best only if E_j < E_best (1 - 1e-12) (ties keep
+ * the wider range).  n_alpha = 1 is q4_quantize_pack's symmetric RTN exactly.
+ *   W        [out, in] fp16 or bf16, 16-byte aligned; `in` a multiple of 8
+ *   group_size one of 8, 16, 32, 64, 128, 256 (else Q4_ERR_UNSUPPORTED),
+ *            dividing `in` (else Q4_ERR_SHAPE)
+ *   n_alpha  1 .. 64 (else Q4_ERR_INVALID_ARG)
+ *   qweight  [out, in/2] uint8, 4-byte aligned; scales [out, in/g] fp16.
+ * The output is a symmetric q4_weight for q4_dequant / q4_gemv / q4_gemm_skinny.
+ * Errors of the summation order are below the tie margin, so the chosen
+ * range matches the CPU reference except on ties within 1e-12.
+ */
+Q4_API q4_status q4_quantize_pack_clip(const void* W, q4_dtype w_dtype, int64_t out, int64_t in,
+                                       int32_t group_size, int32_t n_alpha, uint8_t* qweight,
+                                       void* scales, q4_stream stream);
+
+/*
  * Dequantization W_hat = s * (q - z), [out, in], in fp16, bf16 or fp32.
  * s * (q - z) is exact in fp32; fp16 / bf16 outputs are that value rounded
  * to nearest even.  (ybb.press section 二; arganzheng.life section 二.2.)

@@ -36,7 +36,7 @@ _DT = {torch.float16: Q4_F16, torch.bfloat16: Q4_BF16, torch.float32: Q4_F32}
 ABI_SYMBOLS = (
     "q4_quantize_pack", "q4_dequant", "q4_gemv", "q4_gemm_skinny", "bf16_gemv_ref_bw",
     "q4_sync_status", "q4_status_string", "q4_version", "q4_selftest_wait_timeout",
-    "q4_workspace_bytes", "q4_gemv_noalloc",
+    "q4_workspace_bytes", "q4_gemv_noalloc", "q4_quantize_pack_clip",
 )
 
 
@@ -82,6 +82,7 @@ def load_library(path: str = LIB_PATH):
     W = ctypes.POINTER(_CWeight)
     lib.q4_quantize_pack.argtypes = [P, S, I64, I64, I32, I32, I32, P, P, P, P]
     lib.q4_dequant.argtypes = [W, P, S, P]
+    lib.q4_quantize_pack_clip.argtypes = [P, S, I64, I64, I32, I32, P, P, P]
     lib.q4_gemv.argtypes = [W, P, S, I64, P, S, P, ctypes.c_size_t, P]
     lib.q4_gemm_skinny.argtypes = [W, P, S, I64, P, S, P, ctypes.c_size_t, P]
     lib.q4_gemv_noalloc.argtypes = [W, P, S, I64, P, S, P]
@@ -90,7 +91,8 @@ def load_library(path: str = LIB_PATH):
     lib.bf16_gemv_ref_bw.argtypes = [P, I64, I64, P, I64, P, P]
     lib.q4_sync_status.argtypes = [P]
     lib.q4_selftest_wait_timeout.argtypes = [I64, P]
-    for f in ("q4_quantize_pack", "q4_dequant", "q4_gemv", "q4_gemm_skinny", "q4_gemv_noalloc",
+    for f in ("q4_quantize_pack", "q4_quantize_pack_clip", "q4_dequant", "q4_gemv",
+              "q4_gemm_skinny", "q4_gemv_noalloc",
               "bf16_gemv_ref_bw", "q4_sync_status", "q4_selftest_wait_timeout"):
         getattr(lib, f).restype = S
     lib.q4_status_string.argtypes = [S]
@@ -176,6 +178,27 @@ def q4_quantize_pack(W: torch.Tensor, group_size: int = 128, symmetric: bool = T
                               _stream(stream))
     _check(st, "q4_quantize_pack")
     return Q4Weight(qweight, scales, zeros, out, inn, group_size, bool(symmetric), bits)
+
+
+def q4_quantize_pack_clip(W: torch.Tensor, group_size: int = 128, n_alpha: int = 21,
+                          qweight: torch.Tensor | None = None,
+                          scales: torch.Tensor | None = None, stream=None) -> Q4Weight:
+    """Symmetric INT4 quantization with the per-group range search over
+    n_alpha ranges from max|w| down to 0.8 max|w| (q4.h, q4_quantize_pack_clip)."""
+    lib = load_library()
+    if W.dim() != 2 or W.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("W must be a 2-D fp16 or bf16 tensor")
+    out, inn = W.shape
+    G = inn // group_size if group_size > 0 else 0
+    dev = W.device
+    if qweight is None:
+        qweight = torch.empty(out, inn // 2, dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(out, G, dtype=torch.float16, device=dev)
+    st = lib.q4_quantize_pack_clip(_ptr(W), _DT[W.dtype], out, inn, group_size, n_alpha,
+                                   _ptr(qweight), _ptr(scales), _stream(stream))
+    _check(st, "q4_quantize_pack_clip")
+    return Q4Weight(qweight, scales, None, out, inn, group_size, True, 4)
 
 
 def q4_dequant(w: Q4Weight, out_dtype=torch.float32, W_hat: torch.Tensor | None = None,

@@ -227,6 +227,26 @@ q4_status run_quantize(const void* W, int64_t out, int64_t in, int g, uint8_t* q
     return launch_status(cudaSuccess);
 }
 
+template <bool BF16IN>
+q4_status run_quantize_clip(const void* W, int64_t out, int64_t in, int g, int n,
+                            uint8_t* qweight, __half* scales, cudaStream_t st) {
+    const int sms = sm_count(current_device());
+    const int64_t nchunks = out * in / 8;
+    const int64_t want = (nchunks + 255) / 256;
+    const int blocks = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
+    uint32_t* qw = reinterpret_cast<uint32_t*>(qweight);
+    switch (g) {
+#define Q4_CCASE(GV)                                                                         \
+    case GV:                                                                                 \
+        quantize_pack_clip_kernel<GV, BF16IN><<<blocks, 256, 0, st>>>(W, nchunks, n, qw, scales); \
+        break;
+        Q4_CCASE(8) Q4_CCASE(16) Q4_CCASE(32) Q4_CCASE(64) Q4_CCASE(128) Q4_CCASE(256)
+#undef Q4_CCASE
+        default: return Q4_ERR_UNSUPPORTED;
+    }
+    return launch_status(cudaSuccess);
+}
+
 // ------------------------------------------------------------------ GEMV
 // Tile shape of the small-batch kernels (compile-time tunables).
 #ifndef Q4_GEMV_MT
@@ -566,6 +586,28 @@ q4_status q4_quantize_pack(const void* W, q4_dtype w_dtype, int64_t out, int64_t
                   : run_quantize<true, false>(W, out, in, group_size, qweight, s, z, st);
     return bf ? run_quantize<false, true>(W, out, in, group_size, qweight, s, z, st)
               : run_quantize<false, false>(W, out, in, group_size, qweight, s, z, st);
+}
+
+q4_status q4_quantize_pack_clip(const void* W, q4_dtype w_dtype, int64_t out, int64_t in,
+                                int32_t group_size, int32_t n_alpha, uint8_t* qweight,
+                                void* scales, q4_stream stream) {
+    if (w_dtype != Q4_F16 && w_dtype != Q4_BF16) {
+        return valid_dtype(w_dtype) ? Q4_ERR_UNSUPPORTED : Q4_ERR_INVALID_ARG;
+    }
+    if (n_alpha < 1 || n_alpha > 64) return Q4_ERR_INVALID_ARG;
+    if (out < 0 || in <= 0 || group_size <= 0) return Q4_ERR_SHAPE;
+    if ((group_size & 1) || (in % group_size) != 0 || (in % 8) != 0) return Q4_ERR_SHAPE;
+    if (group_size != 8 && group_size != 16 && group_size != 32 && group_size != 64 &&
+        group_size != 128 && group_size != 256)
+        return Q4_ERR_UNSUPPORTED;
+    if (out == 0) return Q4_OK;
+    if (!W || !qweight || !scales) return Q4_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(qweight, 4) || !aligned(scales, 2)) return Q4_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    __half* s = reinterpret_cast<__half*>(scales);
+    return w_dtype == Q4_BF16
+               ? run_quantize_clip<true>(W, out, in, group_size, n_alpha, qweight, s, st)
+               : run_quantize_clip<false>(W, out, in, group_size, n_alpha, qweight, s, st);
 }
 
 q4_status q4_dequant(const q4_weight* w, void* W_hat, q4_dtype out_dtype, q4_stream stream) {

@@ -124,6 +124,74 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const void* __restri
     }
 }
 
+// Symmetric quantization with a per-group range (clipping) search
+// (arganzheng.life post-training-quantization-gptq-awq-and-rotation section
+// 三.2, 裁剪与舍入的权衡: scan ranges alpha from 0.8 to 1.0 of max|w| and keep
+// the one with the smallest error).  Candidates alpha_j = amax (K - j) / K,
+// K = 5 (n - 1), j = 0 .. n-1; s_j = fp16(amax (K - j) / (7 K)) (the product
+// is exact in fp32, the division IEEE); codes clamp(rne(w / s_j), -7, 7), the
+// section's symmetric grid; error sum (w - s_j q)^2 in fp64, reduced over the
+// group's lanes by butterfly shuffles (every lane holds the same sum and takes
+// the same decision); j replaces the best only if its error is below
+// E_best (1 - 1e-12), so ties keep the wider range.  j = 0 is RTN exactly.
+template <int G, bool BF16IN>
+__global__ void __launch_bounds__(256) quantize_pack_clip_kernel(const void* __restrict__ W,
+                                                                 int64_t nchunks, int n,
+                                                                 uint32_t* __restrict__ qweight,
+                                                                 __half* __restrict__ scales) {
+    constexpr int LANES = G / 8;
+    static_assert(LANES >= 1 && LANES <= 32 && (32 % LANES) == 0, "group must tile a warp");
+    const int lane = threadIdx.x & 31;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int K = 5 * (n - 1);
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+         i - lane < nchunks; i += stride) {
+        const bool active = i < nchunks;
+        float v[8];
+        if (active) {
+            load8_f32<BF16IN>(W, i * 8, v);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = 0.f;
+        }
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(v[e]));
+#pragma unroll
+        for (int off = LANES / 2; off >= 1; off >>= 1)
+            a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+        uint32_t best_packed = 0;
+        __half best_s = __float2half_rn(0.f);
+        double best_e = 0.0;
+        for (int j = 0; j < n; ++j) {
+            const float num = (n == 1) ? a : __fmul_rn(a, static_cast<float>(K - j));
+            const float den = (n == 1) ? 7.0f : static_cast<float>(7 * K);
+            const __half s16 = __float2half_rn(__fdiv_rn(num, den));
+            const float sf = __half2float(s16);
+            uint32_t packed = 0;
+            double e = 0.0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int q = (sf == 0.f) ? 0 : quant_one(v[k], sf, 0.f, -7.f, 7.f);
+                packed |= (static_cast<uint32_t>(q) & 0xFu) << (4 * k);
+                const double d = static_cast<double>(v[k]) - static_cast<double>(sf) * q;
+                e += d * d;
+            }
+#pragma unroll
+            for (int off = LANES / 2; off >= 1; off >>= 1) e += __shfl_xor_sync(0xFFFFFFFFu, e, off);
+            if (j == 0 || (sf != 0.f && e < best_e * (1.0 - 1e-12))) {
+                best_e = e;
+                best_packed = packed;
+                best_s = s16;
+            }
+        }
+        if (active) {
+            qweight[i] = best_packed;
+            if ((lane % LANES) == 0) scales[(i * 8) / G] = best_s;
+        }
+    }
+}
+
 // Generic path: any even group size; one warp per group, element pairs
 // strided over the lanes.
 template <bool SYM, bool BF16IN>

@@ -31,8 +31,8 @@ def _declared_symbols():
 
 def test_header_declares_the_abi():
     names = _declared_symbols()
-    assert {"q4_quantize_pack", "q4_dequant", "q4_gemv", "q4_gemm_skinny",
-            "bf16_gemv_ref_bw", "q4_sync_status", "q4_status_string"} <= names
+    assert {"q4_quantize_pack", "q4_quantize_pack_clip", "q4_dequant", "q4_gemv",
+            "q4_gemm_skinny", "bf16_gemv_ref_bw", "q4_sync_status", "q4_status_string"} <= names
     assert names == set(q4.ABI_SYMBOLS)
 
 
@@ -164,3 +164,27 @@ def test_product_path_has_no_cpu_fallback(tmp_path, monkeypatch):
         mod._lib = saved
     src = open(os.path.join(ROOT, "post_weight_quantization_group_b200", "__init__.py")).read()
     assert "import oracle" not in src and "from oracle" not in src
+
+
+def test_quantize_pack_clip_validation(lib):
+    f = lib.q4_quantize_pack_clip
+    ok = dict(W=A16, dt=q4.Q4_F16, out=8, inn=256, g=128, n=21, q=A16, s=A16)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["W"], a["dt"], a["out"], a["inn"], a["g"], a["n"], a["q"], a["s"], None)
+
+    assert call(n=0) == q4.Q4_ERR_INVALID_ARG
+    assert call(n=65) == q4.Q4_ERR_INVALID_ARG
+    assert call(dt=q4.Q4_F32) == q4.Q4_ERR_UNSUPPORTED
+    assert call(dt=7) == q4.Q4_ERR_INVALID_ARG
+    assert call(g=96) == q4.Q4_ERR_SHAPE            # does not divide 256
+    assert call(g=4, inn=256) == q4.Q4_ERR_UNSUPPORTED
+    assert call(inn=260, g=130) == q4.Q4_ERR_SHAPE  # in not a multiple of 8
+    assert call(out=-1) == q4.Q4_ERR_SHAPE
+    assert call(W=None) == q4.Q4_ERR_INVALID_ARG
+    assert call(s=None) == q4.Q4_ERR_INVALID_ARG
+    assert call(W=A2) == q4.Q4_ERR_ALIGNMENT
+    assert call(q=A2) == q4.Q4_ERR_ALIGNMENT
+    assert call(out=0) == q4.Q4_OK                  # empty: nothing launched

@@ -383,3 +383,90 @@ def test_skinny_consistency():
     ref = x.float() @ q4.q4_dequant(w, torch.float32).T
     rms = ref.pow(2).mean().sqrt()
     assert torch.all((y16 - y32[16:32]).abs() <= 4e-3 * (ref[16:32].abs() + rms))
+
+
+# ------------------------------------------- range (clipping) search quantizer
+
+def _codes(qweight: np.ndarray, inn: int) -> np.ndarray:
+    """Signed codes [out, in] of a symmetric packed matrix."""
+    lo = (qweight & 0xF).astype(np.int32)
+    hi = (qweight >> 4).astype(np.int32)
+    c = np.stack([lo, hi], axis=-1).reshape(qweight.shape[0], inn)
+    return np.where(c >= 8, c - 16, c)
+
+
+def _clip_check(W, g, n, rows=None):
+    """GPU range search against the oracle: each group's scale is one of the
+    oracle's minimum-error candidates (ties within the 1e-12 margin may go
+    either way) and its codes are bit-exact at that scale."""
+    w = q4.q4_quantize_pack_clip(W, g, n)
+    torch.cuda.synchronize()
+    assert q4.q4_sync_status() == q4.Q4_OK
+    rows = np.arange(W.shape[0]) if rows is None else rows
+    rows_t = torch.as_tensor(rows, device=W.device)
+    Wr = _f32(W[rows_t])
+    out, inn = Wr.shape
+    G = inn // g
+    gq = w.qweight[rows_t].cpu().numpy()
+    gs = _np16(w.scales[rows_t])
+    q_ref, s_ref, idx = oracle.quantize_pack_clip(Wr, g, n)
+    same = gs == s_ref
+    # groups where the GPU chose the oracle's scale: codes bit-exact there
+    codes_gpu = _codes(gq, inn).reshape(out, G, g)
+    codes_ref = _codes(q_ref, inn).reshape(out, G, g)
+    assert np.array_equal(codes_gpu[same], codes_ref[same])
+    # any other group must be a tie the margin allows, with consistent codes
+    for r, j in zip(*np.nonzero(~same)):
+        wg = Wr[r, j * g:(j + 1) * g]
+        best, err, s16 = oracle.clip_errors(wg, n)
+        cand = np.nonzero(s16 == gs[r, j])[0]
+        assert cand.size and err[cand].min() <= err[best] * (1 + 1e-9), (r, j)
+        sf = np.float32(np.uint16(gs[r, j]).view(np.float16))
+        exp = np.clip(np.rint(wg / sf), -7, 7) if sf != 0 else np.zeros(g)
+        assert np.array_equal(codes_gpu[r, j], exp.astype(np.int32)), (r, j)
+    return w, float(np.mean(same))
+
+
+@pytest.mark.parametrize("wdtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("kind", ["normal", "t3", "uniform"])
+@pytest.mark.parametrize("g", [8, 32, 64, 128, 256])
+def test_quantize_clip_parity(wdtype, kind, g):
+    W = _weight(kind, 96, 1024, 51).to(wdtype)
+    _, agree = _clip_check(W, g, 21)
+    assert agree > 0.99
+
+
+def test_quantize_clip_single_candidate_is_rtn():
+    W = wl.student_t_weight(300, 2048, 52, device="cuda")
+    a = q4.q4_quantize_pack_clip(W, 128, 1)
+    b = q4.q4_quantize_pack(W, 128, True)
+    assert torch.equal(a.qweight, b.qweight) and torch.equal(a.scales, b.scales)
+
+
+@pytest.mark.parametrize("n", [2, 9, 64])
+def test_quantize_clip_grid_sizes(n):
+    _clip_check(wl.normal_weight(64, 2048, 53 + n, device="cuda"), 128, n)
+
+
+def test_quantize_clip_full_size_sampled_and_lower_error():
+    """70B gate_proj, Student-t(3): sampled rows against the oracle; over the
+    whole matrix the range search lowers the weight error against RTN."""
+    out, inn = wl.LLAMA3_70B["gate_proj"]
+    W = wl.student_t_weight(out, inn, 54, device="cuda")
+    w, _ = _clip_check(W, 128, 21, rows=_sample_rows(out, 64, seed=54))
+    r = q4.q4_quantize_pack(W, 128, True)
+    Wf = W.float()
+    mse_clip = (q4.q4_dequant(w) - Wf).pow(2).mean().item()
+    mse_rtn = (q4.q4_dequant(r) - Wf).pow(2).mean().item()
+    assert mse_clip < 0.9 * mse_rtn
+
+
+def test_quantize_clip_feeds_the_product():
+    W = wl.student_t_weight(700, 2048, 55, device="cuda")
+    w = q4.q4_quantize_pack_clip(W, 64, 21)
+    x = wl.activations(3, 2048, 56, device="cuda")
+    y = q4.q4_gemv(w, x, y_dtype=torch.float32)
+    q_np = w.qweight.cpu().numpy()
+    s_np = _np16(w.scales)
+    y_ref = oracle.gemv(q_np, s_np, None, 700, 2048, 64, True, x.float().cpu().numpy().astype(np.float64))
+    _assert_within(y.cpu().numpy(), y_ref, "clip-quantized product")
