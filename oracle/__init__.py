@@ -78,6 +78,8 @@ def _load():
     lib.oracle_gemv_f64.restype = ctypes.c_int
     lib.oracle_dense_rows_f64.argtypes = [P, I64, I64, P, I64, P, I64, P]
     lib.oracle_dense_rows_f64.restype = ctypes.c_int
+    lib.oracle_quantize_pack_perm.argtypes = [P, I64, I64, I32, I32, P, P, P, P]
+    lib.oracle_quantize_pack_perm.restype = ctypes.c_int
     lib.oracle_clip_search_group.argtypes = [P, I32, I32, P, P]
     lib.oracle_clip_search_group.restype = I32
     lib.oracle_quantize_pack_clip.argtypes = [P, I64, I64, I32, I32, P, P, P]
@@ -159,6 +161,31 @@ def quantize_pack(W: np.ndarray, group_size: int, symmetric: bool):
     if rc != 0:
         raise ValueError("oracle_quantize_pack rejected its arguments")
     return q, s, z
+
+
+def quantize_pack_perm(W: np.ndarray, group_size: int, symmetric: bool, perm: np.ndarray):
+    """Act-order quantization: columns taken in the order perm (groups over
+    that order, codes and scales stored in it).  Same outputs as quantize_pack."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    perm = np.ascontiguousarray(perm, dtype=np.int32)
+    out, inn = W.shape
+    G = inn // group_size
+    q = np.zeros((out, inn // 2), dtype=np.uint8)
+    s = np.zeros((out, G), dtype=np.uint16)
+    z = None if symmetric else np.zeros((out, G), dtype=np.uint16)
+    rc = _load().oracle_quantize_pack_perm(_ptr(W), out, inn, int(group_size), int(bool(symmetric)),
+                                           _ptr(perm), _ptr(q), _ptr(s), _ptr(z))
+    if rc != 0:
+        raise ValueError("oracle_quantize_pack_perm rejected its arguments")
+    return q, s, z
+
+
+def g_idx(perm: np.ndarray, group_size: int) -> np.ndarray:
+    """Group of each original column: g_idx[perm[j]] = j // group_size."""
+    perm = np.asarray(perm, dtype=np.int64)
+    gi = np.empty(perm.size, dtype=np.int32)
+    gi[perm] = np.arange(perm.size) // group_size
+    return gi
 
 
 def quantize_pack_clip(W: np.ndarray, group_size: int, n_alpha: int):

@@ -230,6 +230,31 @@ ORACLE_API int oracle_quantize_pack(const float* W, int64_t out, int64_t in, int
 }
 
 /*
+ * Act-order quantization ("post-training-quantization-gptq-awq-and-rotation"
+ * (arganzheng.life) section 五.3: desc_act quantizes the columns in the
+ * order of decreasing input-channel variance, and the kernels then need a
+ * reorder index g_idx; section 九.2: that reorder is a gather).  The columns
+ * are taken in the order perm[0], perm[1], ...: groups are g consecutive
+ * positions of that order and the codes and scales are stored in it, so
+ *   packed column j  <->  original column perm[j],   g_idx[perm[j]] = j / g.
+ * This is oracle_quantize_pack applied to the column-permuted matrix.
+ */
+ORACLE_API int oracle_quantize_pack_perm(const float* W, int64_t out, int64_t in, int32_t g,
+                                         int32_t symmetric, const int32_t* perm, uint8_t* qweight,
+                                         uint16_t* scales, uint16_t* zeros) {
+    if (in <= 0 || out < 0) return -1;
+    for (int64_t j = 0; j < in; ++j)
+        if (perm[j] < 0 || perm[j] >= in) return -1;
+    float* Wp = (float*)malloc(sizeof(float) * (size_t)(out > 0 ? out : 1) * (size_t)in);
+    if (!Wp) return -1;
+    for (int64_t r = 0; r < out; ++r)
+        for (int64_t j = 0; j < in; ++j) Wp[r * in + j] = W[r * in + perm[j]];
+    const int rc = oracle_quantize_pack(Wp, out, in, g, symmetric, qweight, scales, zeros);
+    free(Wp);
+    return rc;
+}
+
+/*
  * Range (clipping) search of symmetric INT4 group quantization
  * ("post-training-quantization-gptq-awq-and-rotation" (arganzheng.life),
  * section 三.2, 裁剪与舍入的权衡: scan a set of ranges alpha between 0.8 and

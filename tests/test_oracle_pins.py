@@ -442,3 +442,65 @@ def test_clip_search_gaussian_optimum_below_max():
     amax = np.abs(W).max(axis=1) / sigma
     # the floor 0.8 max lies at or above 2.5 sigma: the optimum is below it
     assert np.all(0.8 * amax > 2.5) and np.median(amax) > 3.5
+
+
+# ------------------------------------------------------------- act-order
+# arganzheng.life post-training-quantization-gptq-awq-and-rotation, section
+# 五.3 (desc_act, g_idx) and 九.2 (the reorder is a gather).
+
+@pytest.mark.parametrize("sym", [True, False])
+def test_act_order_identity_is_plain_quantization(sym):
+    W = wl.normal_weight(24, 512, 61).float().numpy()
+    a = oracle.quantize_pack_perm(W, 64, sym, np.arange(512, dtype=np.int32))
+    b = oracle.quantize_pack(W, 64, sym)
+    for x, y in zip(a, b):
+        assert (x is None and y is None) or np.array_equal(x, y)
+
+
+@pytest.mark.parametrize("sym", [True, False])
+def test_act_order_groups_follow_g_idx(sym):
+    """Column k's code and scale are those of group g_idx[k]: each group's
+    scale is the statistic of exactly the columns g_idx assigns to it
+    (checked column by column, without building the permuted matrix)."""
+    rng = np.random.default_rng(62)
+    out, inn, g = 16, 512, 128
+    W = wl.student_t_weight(out, inn, 63).float().numpy()
+    perm = rng.permutation(inn).astype(np.int32)
+    q, s, z = oracle.quantize_pack_perm(W, g, sym, perm)
+    gi = oracle.g_idx(perm, g)
+    assert np.array_equal(np.bincount(gi), np.full(inn // g, g))
+    pos = np.empty(inn, dtype=np.int64)
+    pos[perm] = np.arange(inn)
+    for r in range(out):
+        for t in range(inn // g):
+            cols = np.nonzero(gi == t)[0]
+            wv = W[r, cols]
+            if sym:
+                want = np.float16(np.float32(np.max(np.abs(wv))) / np.float32(7.0))
+            else:
+                want = np.float16(np.float32(np.float32(wv.max()) - np.float32(wv.min())) / np.float32(15.0))
+            assert np.uint16(s[r, t]) == want.view(np.uint16)
+        # dequantised value of every original column from its own position
+        Wh = oracle.dequant(q, s, z, out, inn, g, sym)[r]
+        sf = np.asarray(s[r]).view(np.float16).astype(np.float32)
+        for k in rng.choice(inn, 16, replace=False):
+            j = pos[k]
+            code = oracle.code_at(q, inn, r, int(j), sym)
+            zz = 0.0 if sym else float(np.asarray(z[r, j // g]).view(np.float16))
+            assert Wh[j] == np.float32(sf[j // g] * np.float32(code - zz))
+
+
+def test_act_order_product_is_a_gather():
+    """y = x W_hat^T over original columns equals the product of the stored
+    (permuted) weights with the gathered activations x[:, perm]."""
+    rng = np.random.default_rng(64)
+    out, inn, g = 40, 1024, 128
+    W = wl.normal_weight(out, inn, 65).float().numpy()
+    perm = rng.permutation(inn).astype(np.int32)
+    q, s, _ = oracle.quantize_pack_perm(W, g, True, perm)
+    x = wl.activations(3, inn, 66).float().numpy().astype(np.float64)
+    y_gather = oracle.gemv(q, s, None, out, inn, g, True, x[:, perm])
+    Wp = oracle.dequant(q, s, None, out, inn, g, True).astype(np.float64)
+    W_orig = np.empty_like(Wp)
+    W_orig[:, perm] = Wp
+    assert np.allclose(y_gather, x @ W_orig.T, rtol=1e-12, atol=1e-12)
