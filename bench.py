@@ -218,6 +218,32 @@ def b_sweep(q4, wl, torch, device, stream):
             "B_even": even if even is not None else f"> {SWEEP_B[-1]}"}
 
 
+def act_order_cost(q4, wl, torch, device, stream):
+    """Cost of act order at B = 1 on the 70B down_proj shape (8192 x 28672,
+    sym g128, random column order): the gather of x alone, the product alone
+    on gathered x, and both (q4_gemm_act_order), graph-timed, two weight
+    copies rotating."""
+    out, inn = wl.LLAMA3_70B["down_proj"]
+    g = torch.Generator().manual_seed(90)
+    perm = torch.randperm(inn, generator=g).to(torch.int32).to(device)
+    ws = [q4.q4_quantize_pack_perm(wl.normal_weight(out, inn, 91 + i, device=device), perm, 128, True)
+          for i in range(2)]
+    x = wl.activations(1, inn, 92, device=device)
+    xp = torch.empty_like(x)
+    y = torch.empty(1, out, dtype=torch.bfloat16, device=device)
+    wsp = q4.workspace_for(ws[0], 1, device)
+    t_gather = graph_time_us(torch, lambda i: q4.q4_permute_activations(x, perm, xp), 16, stream)
+    t_prod = graph_time_us(torch, lambda i: q4.q4_gemv(ws[i % 2], xp, y=y, workspace=wsp), 16, stream)
+    t_both = graph_time_us(torch, lambda i: q4.q4_gemm_act_order(ws[i % 2], x, y=y, x_perm=xp,
+                                                                  workspace=wsp), 16, stream)
+    st = q4.q4_sync_status()
+    assert st == q4.Q4_OK, q4.status_string(st)
+    del ws
+    return {"shape": f"{out}x{inn} sym g128 B=1", "gather_us": round(t_gather, 2),
+            "product_us": round(t_prod, 2), "act_order_us": round(t_both, 2),
+            "overhead": round(t_both / t_prod - 1.0, 4)}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -404,6 +430,7 @@ def run_ours(args):
     if rank == 0:
         if world == 1 and not args.no_sweep:
             out["int4_vs_bf16_by_B"] = b_sweep(q4, wl, torch, device, stream)
+            out["act_order"] = act_order_cost(q4, wl, torch, device, stream)
         out["cpu_baseline"] = cpu_baseline() if (world == 1 and not args.no_cpu_baseline) else None
         print(json.dumps(out), flush=True)
     del graph

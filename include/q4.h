@@ -112,6 +112,36 @@ Q4_API q4_status q4_quantize_pack(const void* W, q4_dtype w_dtype, int64_t out, 
                            uint8_t* qweight, void* scales, void* zeros, q4_stream stream);
 
 /*
+ * Act-order quantization ("post-training-quantization-gptq-awq-and-rotation"
+ * (arganzheng.life) section 五.3: GPTQ's desc_act quantizes the columns in the
+ * order of decreasing input-channel variance, and kernels then need the
+ * reorder index g_idx).  The columns are taken in the order perm[0],
+ * perm[1], ...: groups are g consecutive positions of that order and codes,
+ * scales (and zeros) are stored in it, i.e. this is q4_quantize_pack of
+ * W[:, perm]; g_idx[perm[j]] = j / g.  The product of such a weight with x
+ * is the product of the stored weight with x[:, perm]
+ * (q4_permute_activations, then q4_gemv / q4_gemm_skinny).
+ *   perm  int32 [in], a permutation of [0, in), 4-byte aligned; an entry
+ *         outside [0, in) is clamped and the next q4_sync_status returns
+ *         Q4_ERR_INVALID_ARG (nothing is read out of bounds).
+ *   W may be 2-byte aligned; other arguments and errors as q4_quantize_pack.
+ */
+Q4_API q4_status q4_quantize_pack_perm(const void* W, q4_dtype w_dtype, int64_t out, int64_t in,
+                                       int32_t group_size, int32_t bits, int32_t symmetric,
+                                       const int32_t* perm, uint8_t* qweight, void* scales,
+                                       void* zeros, q4_stream stream);
+
+/*
+ * The gather of act order (arganzheng.life section 九.2: the g_idx reorder is
+ * a gather): x_perm[b, j] = x[b, perm[j]] for a [rows, in] fp16 or bf16
+ * matrix.  x 2-byte aligned, x_perm 16-byte aligned, `in` a multiple of 8;
+ * perm as for q4_quantize_pack_perm (out-of-range entries clamped and
+ * reported by q4_sync_status as Q4_ERR_INVALID_ARG).
+ */
+Q4_API q4_status q4_permute_activations(const void* x, q4_dtype x_dtype, int64_t rows, int64_t in,
+                                        const int32_t* perm, void* x_perm, q4_stream stream);
+
+/*
  * Symmetric group-wise INT4 quantization with a per-group range (clipping)
  * search ("post-training-quantization-gptq-awq-and-rotation" (arganzheng.life)
  * section 三.2, 裁剪与舍入的权衡: scan ranges alpha from 0.8 to 1.0 of max|w|
@@ -250,7 +280,8 @@ Q4_API q4_status bf16_gemv_ref_bw(const void* W, int64_t out, int64_t in, const 
 /*
  * Waits for `stream`, then reports the first device-side error recorded
  * since the previous call (Q4_ERR_TIMEOUT when a kernel's bounded wait ran
- * out) or a pending CUDA error (Q4_ERR_CUDA), and clears the record.
+ * out, Q4_ERR_INVALID_ARG when a permutation entry was out of range) or a
+ * pending CUDA error (Q4_ERR_CUDA), and clears the record.
  */
 Q4_API q4_status q4_sync_status(q4_stream stream);
 

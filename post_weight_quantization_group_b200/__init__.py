@@ -36,7 +36,8 @@ _DT = {torch.float16: Q4_F16, torch.bfloat16: Q4_BF16, torch.float32: Q4_F32}
 ABI_SYMBOLS = (
     "q4_quantize_pack", "q4_dequant", "q4_gemv", "q4_gemm_skinny", "bf16_gemv_ref_bw",
     "q4_sync_status", "q4_status_string", "q4_version", "q4_selftest_wait_timeout",
-    "q4_workspace_bytes", "q4_gemv_noalloc", "q4_quantize_pack_clip",
+    "q4_workspace_bytes", "q4_gemv_noalloc", "q4_quantize_pack_clip", "q4_quantize_pack_perm",
+    "q4_permute_activations",
 )
 
 
@@ -83,6 +84,8 @@ def load_library(path: str = LIB_PATH):
     lib.q4_quantize_pack.argtypes = [P, S, I64, I64, I32, I32, I32, P, P, P, P]
     lib.q4_dequant.argtypes = [W, P, S, P]
     lib.q4_quantize_pack_clip.argtypes = [P, S, I64, I64, I32, I32, P, P, P]
+    lib.q4_quantize_pack_perm.argtypes = [P, S, I64, I64, I32, I32, I32, P, P, P, P, P]
+    lib.q4_permute_activations.argtypes = [P, S, I64, I64, P, P, P]
     lib.q4_gemv.argtypes = [W, P, S, I64, P, S, P, ctypes.c_size_t, P]
     lib.q4_gemm_skinny.argtypes = [W, P, S, I64, P, S, P, ctypes.c_size_t, P]
     lib.q4_gemv_noalloc.argtypes = [W, P, S, I64, P, S, P]
@@ -91,7 +94,8 @@ def load_library(path: str = LIB_PATH):
     lib.bf16_gemv_ref_bw.argtypes = [P, I64, I64, P, I64, P, P]
     lib.q4_sync_status.argtypes = [P]
     lib.q4_selftest_wait_timeout.argtypes = [I64, P]
-    for f in ("q4_quantize_pack", "q4_quantize_pack_clip", "q4_dequant", "q4_gemv",
+    for f in ("q4_quantize_pack", "q4_quantize_pack_clip", "q4_quantize_pack_perm",
+              "q4_permute_activations", "q4_dequant", "q4_gemv",
               "q4_gemm_skinny", "q4_gemv_noalloc",
               "bf16_gemv_ref_bw", "q4_sync_status", "q4_selftest_wait_timeout"):
         getattr(lib, f).restype = S
@@ -146,6 +150,7 @@ class Q4Weight:
     group_size: int
     symmetric: bool
     bits: int = 4
+    perm: torch.Tensor | None = None  # act order: stored column j is original column perm[j]
 
     def c_struct(self) -> _CWeight:
         return _CWeight(_ptr(self.qweight), _ptr(self.scales), _ptr(self.zeros), self.out,
@@ -199,6 +204,52 @@ def q4_quantize_pack_clip(W: torch.Tensor, group_size: int = 128, n_alpha: int =
                                    _ptr(qweight), _ptr(scales), _stream(stream))
     _check(st, "q4_quantize_pack_clip")
     return Q4Weight(qweight, scales, None, out, inn, group_size, True, 4)
+
+
+def q4_quantize_pack_perm(W: torch.Tensor, perm: torch.Tensor, group_size: int = 128,
+                          symmetric: bool = True, stream=None) -> Q4Weight:
+    """Act-order quantization: columns taken in the order perm (int32 [in] on
+    the device); the result carries perm for q4_gemm_act_order."""
+    lib = load_library()
+    if W.dim() != 2 or W.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("W must be a 2-D fp16 or bf16 tensor")
+    if perm.dtype != torch.int32 or perm.dim() != 1 or perm.numel() != W.shape[1]:
+        raise ValueError("perm must be int32 [in]")
+    out, inn = W.shape
+    G = inn // group_size if group_size > 0 else 0
+    dev = W.device
+    qweight = torch.empty(out, inn // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(out, G, dtype=torch.float16, device=dev)
+    zeros = None if symmetric else torch.empty(out, G, dtype=torch.float16, device=dev)
+    st = lib.q4_quantize_pack_perm(_ptr(W), _DT[W.dtype], out, inn, group_size, 4, int(symmetric),
+                                   _ptr(perm), _ptr(qweight), _ptr(scales), _ptr(zeros),
+                                   _stream(stream))
+    _check(st, "q4_quantize_pack_perm")
+    return Q4Weight(qweight, scales, zeros, out, inn, group_size, bool(symmetric), 4, perm)
+
+
+def q4_permute_activations(x: torch.Tensor, perm: torch.Tensor, x_perm: torch.Tensor | None = None,
+                           stream=None) -> torch.Tensor:
+    """x_perm[b, j] = x[b, perm[j]] (the act-order gather)."""
+    lib = load_library()
+    if x.dim() != 2:
+        raise ValueError("x must be [rows, in]")
+    if x_perm is None:
+        x_perm = torch.empty_like(x)
+    st = lib.q4_permute_activations(_ptr(x), _DT[x.dtype], x.shape[0], x.shape[1], _ptr(perm),
+                                    _ptr(x_perm), _stream(stream))
+    _check(st, "q4_permute_activations")
+    return x_perm
+
+
+def q4_gemm_act_order(w: Q4Weight, x: torch.Tensor, y: torch.Tensor | None = None, y_dtype=None,
+                      x_perm: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """y = x W_hat^T for an act-order weight: the gather, then the product."""
+    if w.perm is None:
+        raise ValueError("w has no column order (quantize it with q4_quantize_pack_perm)")
+    xp = q4_permute_activations(x, w.perm, x_perm, stream)
+    return q4_gemm_skinny(w, xp, y, y_dtype, workspace, stream)
 
 
 def q4_dequant(w: Q4Weight, out_dtype=torch.float32, W_hat: torch.Tensor | None = None,

@@ -198,7 +198,12 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns) {
 // --------------------------------------------------------- quantize_pack
 template <bool SYM, bool BF16IN>
 q4_status run_quantize(const void* W, int64_t out, int64_t in, int g, uint8_t* qweight,
-                       __half* scales, __half* zeros, cudaStream_t st) {
+                       __half* scales, __half* zeros, cudaStream_t st,
+                       const int32_t* perm = nullptr) {
+    unsigned* status = nullptr;
+    if (perm != nullptr &&
+        cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
+        return Q4_ERR_CUDA;
     const int dev = current_device();
     const int sms = sm_count(dev);
     const int64_t ngroups = out * (in / g);
@@ -213,7 +218,8 @@ q4_status run_quantize(const void* W, int64_t out, int64_t in, int g, uint8_t* q
         switch (g) {
 #define Q4_QCASE(GV)                                                                              \
     case GV:                                                                                      \
-        quantize_pack_kernel<GV, SYM, BF16IN><<<blocks, 256, 0, st>>>(W, nchunks, qw, scales, zeros); \
+        quantize_pack_kernel<GV, SYM, BF16IN><<<blocks, 256, 0, st>>>(W, nchunks, qw, scales, zeros, \
+                                                                     perm, in, status);           \
         break;
             Q4_QCASE(8) Q4_QCASE(16) Q4_QCASE(32) Q4_QCASE(64) Q4_QCASE(128) Q4_QCASE(256)
 #undef Q4_QCASE
@@ -223,7 +229,8 @@ q4_status run_quantize(const void* W, int64_t out, int64_t in, int g, uint8_t* q
     const int64_t want = (ngroups * 32 + 255) / 256;
     const int blocks = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
     quantize_pack_generic_kernel<SYM, BF16IN><<<blocks, 256, 0, st>>>(W, ngroups, g, qweight,
-                                                                      scales, zeros);
+                                                                      scales, zeros, perm, in,
+                                                                      status);
     return launch_status(cudaSuccess);
 }
 
@@ -588,6 +595,55 @@ q4_status q4_quantize_pack(const void* W, q4_dtype w_dtype, int64_t out, int64_t
               : run_quantize<false, false>(W, out, in, group_size, qweight, s, z, st);
 }
 
+q4_status q4_quantize_pack_perm(const void* W, q4_dtype w_dtype, int64_t out, int64_t in,
+                                int32_t group_size, int32_t bits, int32_t symmetric,
+                                const int32_t* perm, uint8_t* qweight, void* scales, void* zeros,
+                                q4_stream stream) {
+    if (w_dtype != Q4_F16 && w_dtype != Q4_BF16) {
+        return valid_dtype(w_dtype) ? Q4_ERR_UNSUPPORTED : Q4_ERR_INVALID_ARG;
+    }
+    if (bits != 4) return Q4_ERR_UNSUPPORTED;
+    if (symmetric != 0 && symmetric != 1) return Q4_ERR_INVALID_ARG;
+    if (out < 0 || in <= 0 || group_size <= 0) return Q4_ERR_SHAPE;
+    if ((group_size & 1) || (in % group_size) != 0 || (in % 8) != 0) return Q4_ERR_SHAPE;
+    if (out == 0) return Q4_OK;
+    if (!W || !qweight || !scales || !perm) return Q4_ERR_INVALID_ARG;
+    if (symmetric ? (zeros != nullptr) : (zeros == nullptr)) return Q4_ERR_INVALID_ARG;
+    if (!aligned(W, 2) || !aligned(qweight, 4) || !aligned(scales, 2) || !aligned(perm, 4) ||
+        (zeros && !aligned(zeros, 2)))
+        return Q4_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    __half* s = reinterpret_cast<__half*>(scales);
+    __half* z = reinterpret_cast<__half*>(zeros);
+    const bool bf = (w_dtype == Q4_BF16);
+    if (symmetric)
+        return bf ? run_quantize<true, true>(W, out, in, group_size, qweight, s, z, st, perm)
+                  : run_quantize<true, false>(W, out, in, group_size, qweight, s, z, st, perm);
+    return bf ? run_quantize<false, true>(W, out, in, group_size, qweight, s, z, st, perm)
+              : run_quantize<false, false>(W, out, in, group_size, qweight, s, z, st, perm);
+}
+
+q4_status q4_permute_activations(const void* x, q4_dtype x_dtype, int64_t rows, int64_t in,
+                                 const int32_t* perm, void* x_perm, q4_stream stream) {
+    if (!valid_dtype(x_dtype)) return Q4_ERR_INVALID_ARG;
+    if (x_dtype == Q4_F32) return Q4_ERR_UNSUPPORTED;
+    if (rows < 0 || in <= 0 || (in % 8) != 0) return Q4_ERR_SHAPE;
+    if (rows == 0) return Q4_OK;
+    if (!x || !perm || !x_perm) return Q4_ERR_INVALID_ARG;
+    if (!aligned(x, 2) || !aligned(perm, 4) || !aligned(x_perm, 16)) return Q4_ERR_ALIGNMENT;
+    unsigned* status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
+        return Q4_ERR_CUDA;
+    const int sms = sm_count(current_device());
+    const int64_t n8 = rows * in / 8;
+    const int64_t want = (n8 + 255) / 256;
+    const int blocks = static_cast<int>(want < 4LL * sms ? want : 4LL * sms);
+    return launch_ex(permute_columns_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, 1,
+                     true, reinterpret_cast<cudaStream_t>(stream),
+                     reinterpret_cast<const uint16_t*>(x), rows, in, perm,
+                     reinterpret_cast<uint16_t*>(x_perm), status);
+}
+
 q4_status q4_quantize_pack_clip(const void* W, q4_dtype w_dtype, int64_t out, int64_t in,
                                 int32_t group_size, int32_t n_alpha, uint8_t* qweight,
                                 void* scales, q4_stream stream) {
@@ -764,6 +820,7 @@ q4_status q4_sync_status(q4_stream stream) {
             noalloc_mark_reclear();
             return Q4_ERR_TIMEOUT;
         }
+        if (h & kStatusBadIndex) return Q4_ERR_INVALID_ARG;
     }
     return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }

@@ -12,7 +12,9 @@ namespace q4dev {
 
 // ---------------------------------------------------------------- status
 // Device-side error word: bit 0 = a bounded wait ran out.
-enum : unsigned { kStatusTimeout = 1u };
+// Bit 1 = an index argument (a column permutation) was out of range; the
+// kernel clamped it and went on.
+enum : unsigned { kStatusTimeout = 1u, kStatusBadIndex = 2u };
 
 // A bounded wait gives up after this many nanoseconds (%globaltimer), sets
 // kStatusTimeout in the status word and lets the kernel finish without

@@ -41,6 +41,35 @@ __device__ __forceinline__ void load8_f32(const void* base, int64_t elem, float 
     }
 }
 
+// Column index perm[c] clamped into [0, in); a bad entry is recorded.
+__device__ __forceinline__ int64_t perm_col(const int32_t* perm, int64_t c, int64_t in,
+                                            unsigned* status) {
+    int64_t k = perm[c];
+    if (k < 0 || k >= in) {
+        atomicOr(status, kStatusBadIndex);
+        k = k < 0 ? 0 : in - 1;
+    }
+    return k;
+}
+
+// Eight consecutive columns c0 .. c0+7 of row r taken through perm
+// (act order): element e is W[r, perm[c0 + e]].
+template <bool BF16IN>
+__device__ __forceinline__ void load8_perm_f32(const void* base, int64_t r, int64_t c0, int64_t in,
+                                               const int32_t* perm, unsigned* status,
+                                               float (&v)[8]) {
+    const uint16_t* w16 = reinterpret_cast<const uint16_t*>(base) + r * in;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const uint16_t b = __ldg(w16 + perm_col(perm, c0 + e, in, status));
+        if constexpr (BF16IN) {
+            v[e] = __uint_as_float(static_cast<uint32_t>(b) << 16);
+        } else {
+            v[e] = __half2float(__ushort_as_half(b));
+        }
+    }
+}
+
 // clamp(rne(w / s) + z, qmin, qmax) with the same fp32 operations as the
 // definition: IEEE division, round half to even, add z, clamp (NaN -> qmin).
 __device__ __forceinline__ int quant_one(float w, float s, float z, float qmin, float qmax) {
@@ -52,12 +81,16 @@ __device__ __forceinline__ int quant_one(float w, float s, float z, float qmin, 
 
 // Fast path: group size G in {8, 16, 32, 64, 128, 256}.  n16 = number of
 // 8-element chunks = out*in/8.
+// With perm (act order, may be null) the columns are read through it: the
+// quantized matrix is W[:, perm] (in = row length, for the gather).
 template <int G, bool SYM, bool BF16IN>
 __global__ void __launch_bounds__(256) quantize_pack_kernel(const void* __restrict__ W,
                                                             int64_t nchunks,
                                                             uint32_t* __restrict__ qweight,
                                                             __half* __restrict__ scales,
-                                                            __half* __restrict__ zeros) {
+                                                            __half* __restrict__ zeros,
+                                                            const int32_t* __restrict__ perm,
+                                                            int64_t in, unsigned* status) {
     constexpr int LANES = G / 8;  // lanes per group
     static_assert(LANES >= 1 && LANES <= 32 && (32 % LANES) == 0, "group must tile a warp");
     const int lane = threadIdx.x & 31;
@@ -67,7 +100,10 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const void* __restri
         const bool active = i < nchunks;
         float v[8];
         if (active) {
-            load8_f32<BF16IN>(W, i * 8, v);
+            if (perm != nullptr)
+                load8_perm_f32<BF16IN>(W, (i * 8) / in, (i * 8) % in, in, perm, status, v);
+            else
+                load8_f32<BF16IN>(W, i * 8, v);
         } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e) v[e] = 0.f;
@@ -197,13 +233,16 @@ __global__ void __launch_bounds__(256) quantize_pack_clip_kernel(const void* __r
 template <bool SYM, bool BF16IN>
 __global__ void __launch_bounds__(256) quantize_pack_generic_kernel(
     const void* __restrict__ W, int64_t ngroups, int g, uint8_t* __restrict__ qweight,
-    __half* __restrict__ scales, __half* __restrict__ zeros) {
+    __half* __restrict__ scales, __half* __restrict__ zeros, const int32_t* __restrict__ perm,
+    int64_t in, unsigned* status) {
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     const uint16_t* w16 = reinterpret_cast<const uint16_t*>(W);
     auto ld = [&](int64_t e) -> float {
-        const uint16_t b = w16[e];
+        // element e of the (column-permuted, with perm) matrix
+        const uint16_t b = perm != nullptr ? w16[(e / in) * in + perm_col(perm, e % in, in, status)]
+                                           : w16[e];
         if constexpr (BF16IN) {
             return __uint_as_float(static_cast<uint32_t>(b) << 16);
         } else {
@@ -321,6 +360,36 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict
             v[e] = __fmul_rn(s, q);
         }
         store8<OutT>(W_hat + e0, v);
+    }
+}
+
+// Activations gathered into the act order: x_perm[b, j] = x[b, perm[j]]
+// (arganzheng.life section 九.2: the g_idx reorder is a gather); one thread
+// per 8 outputs (16-byte store).
+__global__ void __launch_bounds__(256) permute_columns_kernel(const uint16_t* __restrict__ x,
+                                                              int64_t rows, int64_t in,
+                                                              const int32_t* __restrict__ perm,
+                                                              uint16_t* __restrict__ xo,
+                                                              unsigned* status) {
+    // launched as a programmatic dependent: the next kernel (the product) may
+    // start and prefetch its weights at once; x is read only after the
+    // preceding kernel has completed
+    grid_launch_dependents();
+    grid_dependency_wait();
+    const int64_t n8 = rows * in / 8;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+         i += stride) {
+        const int64_t r = (i * 8) / in, c0 = (i * 8) % in;
+        uint16_t o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = __ldg(x + r * in + perm_col(perm, c0 + e, in, status));
+        uint4 v;
+        v.x = o[0] | (static_cast<uint32_t>(o[1]) << 16);
+        v.y = o[2] | (static_cast<uint32_t>(o[3]) << 16);
+        v.z = o[4] | (static_cast<uint32_t>(o[5]) << 16);
+        v.w = o[6] | (static_cast<uint32_t>(o[7]) << 16);
+        *reinterpret_cast<uint4*>(xo + i * 8) = v;
     }
 }
 

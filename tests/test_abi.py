@@ -188,3 +188,27 @@ def test_quantize_pack_clip_validation(lib):
     assert call(W=A2) == q4.Q4_ERR_ALIGNMENT
     assert call(q=A2) == q4.Q4_ERR_ALIGNMENT
     assert call(out=0) == q4.Q4_OK                  # empty: nothing launched
+
+
+def test_act_order_validation(lib):
+    f = lib.q4_quantize_pack_perm
+    ok = dict(W=A16, dt=q4.Q4_F16, out=8, inn=256, g=128, bits=4, sym=1, perm=A16, q=A16, s=A16, z=None)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["W"], a["dt"], a["out"], a["inn"], a["g"], a["bits"], a["sym"], a["perm"],
+                 a["q"], a["s"], a["z"], None)
+
+    assert call(perm=None) == q4.Q4_ERR_INVALID_ARG
+    assert call(perm=A2) == q4.Q4_ERR_ALIGNMENT
+    assert call(bits=8) == q4.Q4_ERR_UNSUPPORTED
+    assert call(g=96) == q4.Q4_ERR_SHAPE
+    assert call(sym=0) == q4.Q4_ERR_INVALID_ARG      # zeros missing
+    assert call(out=0) == q4.Q4_OK
+    p = lib.q4_permute_activations
+    assert p(A16, q4.Q4_BF16, 2, 100, A16, A16, None) == q4.Q4_ERR_SHAPE
+    assert p(A16, q4.Q4_F32, 2, 128, A16, A16, None) == q4.Q4_ERR_UNSUPPORTED
+    assert p(None, q4.Q4_BF16, 2, 128, A16, A16, None) == q4.Q4_ERR_INVALID_ARG
+    assert p(A16, q4.Q4_BF16, 2, 128, A16, A2, None) == q4.Q4_ERR_ALIGNMENT
+    assert p(A16, q4.Q4_BF16, 0, 128, A16, A16, None) == q4.Q4_OK

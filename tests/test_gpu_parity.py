@@ -470,3 +470,71 @@ def test_quantize_clip_feeds_the_product():
     s_np = _np16(w.scales)
     y_ref = oracle.gemv(q_np, s_np, None, 700, 2048, 64, True, x.float().cpu().numpy().astype(np.float64))
     _assert_within(y.cpu().numpy(), y_ref, "clip-quantized product")
+
+
+# ------------------------------------------------------------ act order
+
+def _variance_order(inn, seed):
+    """Columns by decreasing variance of synthetic activations with outlier
+    channels (desc_act orders by the Hessian diagonal, the input variance)."""
+    x = wl.activations(256, inn, seed, n_outliers=8, outlier_seed=seed + 1).float()
+    return torch.argsort(x.var(dim=0), descending=True).to(torch.int32)
+
+
+@pytest.mark.parametrize("order", ["random", "variance"])
+@pytest.mark.parametrize("sym", [True, False])
+@pytest.mark.parametrize("wdtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("g", [32, 128, 96])
+def test_act_order_quantize_bit_exact(order, sym, wdtype, g):
+    inn = 1152  # multiple of 32, 96 and 128... and of 8
+    inn = 1536 if g == 128 else inn
+    W = wl.student_t_weight(200, inn, 71, device="cuda").to(wdtype)
+    if order == "random":
+        perm = torch.randperm(inn, generator=torch.Generator().manual_seed(72)).to(torch.int32)
+    else:
+        perm = _variance_order(inn, 73)
+    w = q4.q4_quantize_pack_perm(W, perm.cuda(), g, sym)
+    torch.cuda.synchronize()
+    assert q4.q4_sync_status() == q4.Q4_OK
+    q_ref, s_ref, z_ref = oracle.quantize_pack_perm(_f32(W), g, sym, perm.numpy())
+    assert np.array_equal(w.qweight.cpu().numpy(), q_ref)
+    assert np.array_equal(_np16(w.scales), s_ref)
+    if not sym:
+        assert np.array_equal(_np16(w.zeros), z_ref)
+
+
+def test_act_order_identity_and_gather():
+    W = wl.normal_weight(128, 1024, 74, device="cuda")
+    ident = torch.arange(1024, dtype=torch.int32, device="cuda")
+    a = q4.q4_quantize_pack_perm(W, ident, 128, True)
+    b = q4.q4_quantize_pack(W, 128, True)
+    assert torch.equal(a.qweight, b.qweight) and torch.equal(a.scales, b.scales)
+    x = wl.activations(5, 1024, 75, device="cuda")
+    perm = torch.randperm(1024, generator=torch.Generator().manual_seed(76)).to(torch.int32).cuda()
+    assert torch.equal(q4.q4_permute_activations(x, perm), x[:, perm.long()])
+
+
+@pytest.mark.parametrize("B", [1, 5, 16, 40])
+def test_act_order_product(B):
+    out, inn, g = 700, 2048, 128
+    W = wl.student_t_weight(out, inn, 77, device="cuda")
+    perm = _variance_order(inn, 78)
+    w = q4.q4_quantize_pack_perm(W, perm.cuda(), g, True)
+    x = wl.activations(B, inn, 79, n_outliers=8, outlier_seed=74, device="cuda")
+    y = q4.q4_gemm_act_order(w, x, y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert q4.q4_sync_status() == q4.Q4_OK
+    q_ref, s_ref, _ = oracle.quantize_pack_perm(_f32(W), g, True, perm.numpy())
+    xn = x.float().cpu().numpy().astype(np.float64)
+    y_ref = oracle.gemv(q_ref, s_ref, None, out, inn, g, True, xn[:, perm.numpy()])
+    _assert_within(y.cpu().numpy(), y_ref, f"act-order B{B}")
+
+
+def test_act_order_bad_index_is_reported():
+    W = wl.normal_weight(64, 256, 80, device="cuda")
+    perm = torch.arange(256, dtype=torch.int32, device="cuda")
+    perm[17] = 9999
+    q4.q4_quantize_pack_perm(W, perm, 128, True)
+    assert q4.q4_sync_status() == q4.Q4_ERR_INVALID_ARG
+    assert q4.q4_sync_status() == q4.Q4_OK
+    _gemv_case(256, 1024, 128, True, 2, torch.bfloat16)  # still usable
