@@ -83,6 +83,11 @@ def _load():
     lib.oracle_clip_search_group.argtypes = [P, I32, I32, P, P]
     lib.oracle_clip_search_group.restype = I32
     lib.oracle_quantize_pack_clip.argtypes = [P, I64, I64, I32, I32, P, P, P]
+    lib.oracle_q8_quantize_per_channel.argtypes = [P, I64, I64, P, P]
+    lib.oracle_q8_dequant_f32.argtypes = [P, P, I64, I64, P]
+    lib.oracle_q8_gemv_rows_f64.argtypes = [P, P, I64, I64, P, I64, P, I64, P]
+    lib.oracle_kv_quantize_int8.argtypes = [P, I64, I64, I32, P, P]
+    lib.oracle_kv_dequant_int8.argtypes = [P, P, I64, I64, I32, P]
     lib.oracle_quantize_pack_clip.restype = ctypes.c_int
     _lib = lib
     return lib
@@ -268,3 +273,87 @@ def dense(W: np.ndarray, x: np.ndarray, rows=None) -> np.ndarray:
     if rc != 0:
         raise ValueError("oracle_dense_rows_f64 rejected its arguments")
     return y
+
+
+# ------------------------------------------------ per-channel INT8 weights
+
+def q8_quantize_per_channel(W: np.ndarray):
+    """W: [out, in] float32.  Returns (q int8 [out, in], scales float32 [out])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    out, inn = W.shape
+    q = np.zeros((out, inn), dtype=np.int8)
+    s = np.zeros(out, dtype=np.float32)
+    if _load().oracle_q8_quantize_per_channel(_ptr(W), out, inn, _ptr(q), _ptr(s)) != 0:
+        raise ValueError("oracle_q8_quantize_per_channel rejected its arguments")
+    return q, s
+
+
+def q8_dequant(q: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """W_hat [out, in] float32 = q * s (one fp32 multiplication)."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    out, inn = q.shape
+    W_hat = np.empty((out, inn), dtype=np.float32)
+    if _load().oracle_q8_dequant_f32(_ptr(q), _ptr(scales), out, inn, _ptr(W_hat)) != 0:
+        raise ValueError("oracle_q8_dequant_f32 rejected its arguments")
+    return W_hat
+
+
+def q8_gemv(q: np.ndarray, scales: np.ndarray, x: np.ndarray, rows=None) -> np.ndarray:
+    """y [B, len(rows)] fp64 = s[r] * sum_k q[r, k] x[b, k] over the given rows."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    out, inn = q.shape
+    x = np.ascontiguousarray(np.atleast_2d(x), dtype=np.float64)
+    B = x.shape[0]
+    if rows is None:
+        rows = np.arange(out, dtype=np.int64)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    y = np.empty((B, rows.shape[0]), dtype=np.float64)
+    if _load().oracle_q8_gemv_rows_f64(_ptr(q), _ptr(scales), out, inn, _ptr(x), B, _ptr(rows),
+                                       rows.shape[0], _ptr(y)) != 0:
+        raise ValueError("oracle_q8_gemv_rows_f64 rejected its arguments")
+    return y
+
+
+# ------------------------------------------------------------- KV cache
+
+def kv_quantize_int8(kv: np.ndarray, is_bf16: bool):
+    """kv: [..., head_dim] float32 (exact values of an fp16 / bf16 cache).
+
+    Returns (codes int8 [..., head_dim], scales uint16 bits of the cache
+    type [...]), one scale per row of head_dim values."""
+    kv = np.ascontiguousarray(kv, dtype=np.float32)
+    d = kv.shape[-1]
+    rows = kv.size // d
+    codes = np.zeros(kv.shape, dtype=np.int8)
+    scales = np.zeros(kv.shape[:-1], dtype=np.uint16)
+    if _load().oracle_kv_quantize_int8(_ptr(kv), rows, d, int(bool(is_bf16)), _ptr(codes),
+                                       _ptr(scales)) != 0:
+        raise ValueError("oracle_kv_quantize_int8 rejected its arguments")
+    return codes, scales
+
+
+def kv_dequant_int8(codes: np.ndarray, scales: np.ndarray, is_bf16: bool) -> np.ndarray:
+    """uint16 bits of the cache type, q * s rounded once."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    d = codes.shape[-1]
+    out = np.zeros(codes.shape, dtype=np.uint16)
+    if _load().oracle_kv_dequant_int8(_ptr(codes), _ptr(scales), codes.size // d, d,
+                                      int(bool(is_bf16)), _ptr(out)) != 0:
+        raise ValueError("oracle_kv_dequant_int8 rejected its arguments")
+    return out
+
+
+def kv_quantize_int4(kv: np.ndarray, group_size: int):
+    """INT4 group quantization of a KV cache along head_dim ("压缩算法"
+    section 7.4.1.2, quantize_kv_cache_int4): the symmetric group quantizer
+    (s = amax / 7, codes in [-8, 7], two codes per byte) on the rows of
+    head_dim values.  Returns (packed uint8 [..., head_dim/2], scales uint16
+    fp16 bits [..., head_dim/group_size])."""
+    kv = np.ascontiguousarray(kv, dtype=np.float32)
+    d = kv.shape[-1]
+    q, s, _ = quantize_pack(kv.reshape(-1, d), group_size, True)
+    lead = kv.shape[:-1]
+    return q.reshape(*lead, d // 2), s.reshape(*lead, d // group_size)

@@ -31,6 +31,10 @@
  *  - two 4-bit codes per byte: "压缩算法" section 7.4.1.2 (pack_int4).
  *  - the decode product y = x W^T of the dequantised weights:
  *    arganzheng.life section 二.1 ([B,k] x [k,n] decode GEMM) and 二.3.
+ *  - per-output-channel INT8 weights, s = max(amax, 1e-6) / 127, codes in
+ *    [-127, 127]: charles2530.github.io, section 13 (快速代码示例).
+ *  - INT8 KV cache, one scale per token row of head_dim values, codes in
+ *    [-128, 127], and its dequantization: "压缩算法" section 7.4.1.1.
  *
  * Readings taken where the pages leave a step open:
  *  - the scale is computed in fp32 (IEEE division), stored as fp16, and the
@@ -426,6 +430,116 @@ ORACLE_API int oracle_dense_rows_f64(const float* W, int64_t out, int64_t in, co
             for (int64_t k = 0; k < in; ++k) acc += (double)W[r * in + k] * x[b * in + k];
             y[b * nrows + i] = acc;
         }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------- per-channel INT8 weights */
+
+/*
+ * Per-output-channel INT8 weight quantization ("量化：PTQ、GPTQ、AWQ 与
+ * SmoothQuant" (charles2530.github.io), section 13, 快速代码示例
+ * per_channel_int8_quant): one scale per row,
+ *   s[r] = max(max_k |W[r, k]|, eps) / 127,   eps = 1e-6,
+ *   q[r, k] = clamp(rne(W[r, k] / s[r]), -127, 127)   (int8),
+ *   w_hat = q * s.
+ * All in fp32 (the page's w is a float tensor), IEEE division, RNE.
+ */
+ORACLE_API int oracle_q8_quantize_per_channel(const float* W, int64_t out, int64_t in,
+                                              int8_t* q, float* scales) {
+    if (out < 0 || in <= 0) return -1;
+    const float eps = 1e-6f;
+    for (int64_t r = 0; r < out; ++r) {
+        const float* w = W + r * in;
+        float a = 0.0f;
+        for (int64_t k = 0; k < in; ++k) {
+            float m = fabsf(w[k]);
+            if (m > a) a = m;
+        }
+        if (a < eps) a = eps;                    /* clamp_min(eps) */
+        const float s = a / 127.0f;
+        scales[r] = s;
+        for (int64_t k = 0; k < in; ++k)
+            q[r * in + k] = (int8_t)oracle_quantize_value(w[k], s, 0, -127, 127);
+    }
+    return 0;
+}
+
+/* w_hat[r, k] = q[r, k] * s[r], one fp32 multiplication. */
+ORACLE_API int oracle_q8_dequant_f32(const int8_t* q, const float* scales, int64_t out,
+                                     int64_t in, float* W_hat) {
+    if (out < 0 || in <= 0) return -1;
+    for (int64_t r = 0; r < out; ++r)
+        for (int64_t k = 0; k < in; ++k) W_hat[r * in + k] = (float)q[r * in + k] * scales[r];
+    return 0;
+}
+
+/*
+ * y[b, i] = s[rows[i]] * sum_k q[rows[i], k] * x[b, k] in fp64 (the W8A16
+ * decode product of the dequantised per-channel weights).
+ */
+ORACLE_API int oracle_q8_gemv_rows_f64(const int8_t* q, const float* scales, int64_t out,
+                                       int64_t in, const double* x, int64_t B,
+                                       const int64_t* rows, int64_t nrows, double* y) {
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t r = rows[i];
+        if (r < 0 || r >= out) return -1;
+        for (int64_t b = 0; b < B; ++b) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < in; ++k) acc += (double)q[r * in + k] * x[b * in + k];
+            y[b * nrows + i] = (double)scales[r] * acc;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------- INT8 KV cache */
+
+static uint16_t to_cache_dtype(float f, int is_bf16) {
+    return is_bf16 ? oracle_f32_to_bf16(f) : oracle_f32_to_f16(f);
+}
+static float from_cache_dtype(uint16_t h, int is_bf16) {
+    return is_bf16 ? oracle_bf16_to_f32(h) : oracle_f16_to_f32(h);
+}
+
+/*
+ * Symmetric INT8 quantization of a KV cache [batch, heads, seq, head_dim]
+ * along head_dim ("压缩算法" (cs-knowledge-wiki), section 7.4.1.1,
+ * quantize_kv_cache_int8 with its default axis = -1): one scale per
+ * (batch, head, token) row of head_dim values,
+ *   s = max |x| / 127  (stored in the cache's 16-bit type),
+ *   q = clamp(rne(x / s), -128, 127),
+ * and the dequantization q * s rounded to the cache type
+ * (dequantize_kv_cache_int8).  rows = batch * heads * seq, row-major.
+ * Readings: fp32 arithmetic with the stored scale (as for the weights); a
+ * row whose stored scale is 0 gets codes 0.
+ */
+ORACLE_API int oracle_kv_quantize_int8(const float* kv, int64_t rows, int64_t d, int32_t is_bf16,
+                                       int8_t* codes, uint16_t* scales) {
+    if (rows < 0 || d <= 0) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        const float* v = kv + r * d;
+        float a = 0.0f;
+        for (int64_t k = 0; k < d; ++k) {
+            float m = fabsf(v[k]);
+            if (m > a) a = m;
+        }
+        const uint16_t sb = to_cache_dtype(a / 127.0f, is_bf16);
+        const float s = from_cache_dtype(sb, is_bf16);
+        scales[r] = sb;
+        for (int64_t k = 0; k < d; ++k)
+            codes[r * d + k] = (int8_t)(s == 0.0f ? 0 : oracle_quantize_value(v[k], s, 0, -128, 127));
+    }
+    return 0;
+}
+
+ORACLE_API int oracle_kv_dequant_int8(const int8_t* codes, const uint16_t* scales, int64_t rows,
+                                      int64_t d, int32_t is_bf16, uint16_t* out) {
+    if (rows < 0 || d <= 0) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        const float s = from_cache_dtype(scales[r], is_bf16);
+        for (int64_t k = 0; k < d; ++k)
+            out[r * d + k] = to_cache_dtype((float)codes[r * d + k] * s, is_bf16);
     }
     return 0;
 }
