@@ -244,6 +244,68 @@ def act_order_cost(q4, wl, torch, device, stream):
             "overhead": round(t_both / t_prod - 1.0, 4)}
 
 
+def w8a16_cost(q4, wl, torch, device, stream, hbm_peak):
+    """Per-channel INT8 W8A16 product (q8_gemv) on the Llama-3-70B down_proj
+    and gate_proj shapes at B = 1 and 8, beside the INT4 product (sym g128)
+    of the same shape: graph-timed, two weight copies rotating so no call finds
+    its weights in L2.  Algorithmic bytes: codes + fp32 row scales + x + y."""
+    res = {}
+    for name in ("down_proj", "gate_proj"):
+        out, inn = wl.LLAMA3_70B[name]
+        w8 = [q4.q8_quantize_per_channel(wl.normal_weight(out, inn, 60 + i, device=device).to(torch.bfloat16))
+              for i in range(2)]
+        w4 = [q4.q4_quantize_pack(wl.normal_weight(out, inn, 60 + i, device=device), 128, True)
+              for i in range(2)]
+        for B in (1, 8):
+            x = wl.activations(B, inn, 61, device=device)
+            y = torch.empty(B, out, dtype=torch.bfloat16, device=device)
+            wsp = q4._shared_workspace(int(q4.load_library().q8_workspace_bytes(out, inn, B)), device)
+            t8 = graph_time_us(torch, lambda i: q4.q8_gemv(w8[i % 2], x, y=y, workspace=wsp), 16, stream)
+            wsp4 = q4.workspace_for(w4[0], B, device)
+            t4 = graph_time_us(torch, lambda i: q4.q4_gemv(w4[i % 2], x, y=y, workspace=wsp4), 16, stream)
+            b8 = out * inn + out * 4 + B * inn * 2 + B * out * 2
+            res[f"{name}_B{B}"] = {"shape": f"{out}x{inn}", "q8_us": round(t8, 2),
+                                   "q8_gbs": round(b8 / t8 / 1e3, 1),
+                                   "q8_frac_of_measured_hbm": round(b8 / t8 / 1e3 / hbm_peak, 4),
+                                   "q4_g128_us": round(t4, 2)}
+        del w8, w4
+    st = q4.q4_sync_status()
+    assert st == q4.Q4_OK, q4.status_string(st)
+    return res
+
+
+def kv_cache_cost(q4, wl, torch, device, stream, hbm_peak):
+    """INT8 and INT4 (group 128) quantization of one Llama-3-70B layer's K
+    cache at 32768 tokens ([1, 8, 32768, 128] bf16, 67 MB), and the INT8
+    dequantization: graph-timed over four rotating caches (268 MB > L2).
+    Algorithmic bytes: cache read + codes + scales written (dequant: the
+    reverse)."""
+    shape = (1, wl.LLAMA3_70B_KV_HEADS, 32768, wl.LLAMA3_70B_HEAD_DIM)
+    caches = [wl.kv_cache(*shape, seed=70 + i, dtype=torch.bfloat16, device=device) for i in range(4)]
+    n = caches[0].numel()
+    rows = n // shape[-1]
+    c8 = [torch.empty(shape, dtype=torch.int8, device=device) for _ in range(4)]
+    s8 = [torch.empty(shape[:-1], dtype=torch.bfloat16, device=device) for _ in range(4)]
+    p4 = [torch.empty(shape[:-1] + (shape[-1] // 2,), dtype=torch.uint8, device=device) for _ in range(4)]
+    s4 = [torch.empty(shape[:-1] + (1,), dtype=torch.float16, device=device) for _ in range(4)]
+    d8 = [torch.empty(shape, dtype=torch.bfloat16, device=device) for _ in range(4)]
+    t_q8 = graph_time_us(torch, lambda i: q4.kv_quantize_int8(caches[i % 4], c8[i % 4], s8[i % 4]), 16, stream)
+    t_q4 = graph_time_us(torch, lambda i: q4.kv_quantize_int4(caches[i % 4], 128, p4[i % 4], s4[i % 4]), 16, stream)
+    t_d8 = graph_time_us(torch, lambda i: q4.kv_dequant_int8(c8[i % 4], s8[i % 4], d8[i % 4]), 16, stream)
+    st = q4.q4_sync_status()
+    assert st == q4.Q4_OK, q4.status_string(st)
+    b_q8 = 2 * n + n + 2 * rows
+    b_q4 = 2 * n + n // 2 + 2 * rows
+    gbs = lambda b, t: round(b / t / 1e3, 1)
+    return {"shape": "x".join(map(str, shape)) + " bf16",
+            "int8_quantize_us": round(t_q8, 2), "int8_quantize_gbs": gbs(b_q8, t_q8),
+            "int8_quantize_frac": round(b_q8 / t_q8 / 1e3 / hbm_peak, 4),
+            "int4_g128_quantize_us": round(t_q4, 2), "int4_quantize_gbs": gbs(b_q4, t_q4),
+            "int4_quantize_frac": round(b_q4 / t_q4 / 1e3 / hbm_peak, 4),
+            "int8_dequant_us": round(t_d8, 2), "int8_dequant_gbs": gbs(b_q8, t_d8),
+            "int8_dequant_frac": round(b_q8 / t_d8 / 1e3 / hbm_peak, 4)}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -431,6 +493,8 @@ def run_ours(args):
         if world == 1 and not args.no_sweep:
             out["int4_vs_bf16_by_B"] = b_sweep(q4, wl, torch, device, stream)
             out["act_order"] = act_order_cost(q4, wl, torch, device, stream)
+            out["w8a16"] = w8a16_cost(q4, wl, torch, device, stream, peak)
+            out["kv_cache"] = kv_cache_cost(q4, wl, torch, device, stream, peak)
         out["cpu_baseline"] = cpu_baseline() if (world == 1 and not args.no_cpu_baseline) else None
         print(json.dumps(out), flush=True)
     del graph

@@ -277,6 +277,91 @@ Q4_API q4_status q4_gemv_noalloc(const q4_weight* w, const void* x, q4_dtype x_d
 Q4_API q4_status bf16_gemv_ref_bw(const void* W, int64_t out, int64_t in, const void* x, int64_t B,
                            void* y, q4_stream stream);
 
+/* ------------------------------------------------ per-channel INT8 weights
+ *
+ * "量化：PTQ、GPTQ、AWQ 与 SmoothQuant" (charles2530.github.io), section 13
+ * (快速代码示例, per_channel_int8_quant): one scale per output row of
+ * W [out, in], in fp32 with IEEE divisions and round-half-to-even,
+ *   s[r] = max(max_k |W[r, k]|, 1e-6) / 127,   q = clamp(rne(W / s), -127, 127),
+ * and w_hat = q * s.
+ *
+ *   W        [out, in] fp16 or bf16 (fp32: Q4_ERR_UNSUPPORTED), 16-byte aligned
+ *   qweight  [out, in] int8, row-major, 16-byte aligned (written)
+ *   scales   [out] fp32, 4-byte aligned (written)
+ *   in       a multiple of 16 (else Q4_ERR_SHAPE); out == 0 is a no-op
+ * The caller owns every buffer.  Asynchronous on `stream`.
+ */
+Q4_API q4_status q8_quantize_per_channel(const void* W, q4_dtype w_dtype, int64_t out, int64_t in,
+                                         int8_t* qweight, float* scales, q4_stream stream);
+
+/* W_hat[r, k] = q[r, k] * s[r] (one fp32 product), written as out_dtype
+ * (rounded to nearest even for fp16 / bf16).  W_hat [out, in], 16-byte
+ * aligned; same shape rules as q8_quantize_per_channel. */
+Q4_API q4_status q8_dequant(const int8_t* qweight, const float* scales, int64_t out, int64_t in,
+                            void* W_hat, q4_dtype out_dtype, q4_stream stream);
+
+/* Workspace bytes q8_gemv needs for this shape (0 for invalid arguments).
+ * The layout is that of q4_gemv's workspace (a zeroed counter region, then
+ * partial slots), so one buffer of the larger size serves both. */
+Q4_API size_t q8_workspace_bytes(int64_t out, int64_t in, int64_t B);
+
+/*
+ * W8A16 decode product y[b, r] = s[r] * sum_k q[r, k] * x[b, k] for
+ * 1 <= B <= 8 (else Q4_ERR_SHAPE): a persistent stream-K kernel on 16-bit
+ * tensor cores with the codes converted exactly on chip and fp32
+ * accumulation; the row scale multiplies the finished sum.
+ *   x   [B, in] fp16 or bf16, 16-byte aligned
+ *   y   [B, out] x_dtype or fp32, 16-byte aligned
+ *   in  a multiple of 16, at most 2^30; out at most 65535 * 128
+ *   workspace  >= q8_workspace_bytes(out, in, B) bytes, 256-byte aligned,
+ *              zero-filled once before first use (the kernel leaves it so)
+ * Deterministic: the result does not depend on timing.  A bounded wait that
+ * runs out is reported by q4_sync_status as Q4_ERR_TIMEOUT.
+ */
+Q4_API q4_status q8_gemv(const int8_t* qweight, const float* scales, int64_t out, int64_t in,
+                         const void* x, q4_dtype x_dtype, int64_t B, void* y, q4_dtype y_dtype,
+                         void* workspace, size_t workspace_bytes, q4_stream stream);
+
+/* --------------------------------------------------------------- KV cache
+ *
+ * A KV cache [batch, heads, seq, head_dim] in fp16 or bf16 is passed as
+ * rows = batch * heads * seq contiguous rows of head_dim values.
+ *
+ * INT8 ("压缩算法" (cs-knowledge-wiki), section 7.4.1.1,
+ * quantize_kv_cache_int8 / dequantize_kv_cache_int8 along the last axis):
+ * one scale per row, stored in the cache's own type,
+ *   s = cache_type(max |x| / 127),   q = clamp(rne(x / s), -128, 127),
+ * in fp32 with the stored scale; a row whose stored scale is 0 gets codes 0.
+ *   kv      [rows, head_dim], 16-byte aligned
+ *   codes   [rows, head_dim] int8, 16-byte aligned (written)
+ *   scales  [rows] in the cache type, 2-byte aligned (written)
+ *   head_dim a multiple of 8 in [8, 512] (else Q4_ERR_SHAPE)
+ */
+Q4_API q4_status kv_quantize_int8(const void* kv, q4_dtype dtype, int64_t rows, int64_t head_dim,
+                                  int8_t* codes, void* scales, q4_stream stream);
+
+/* out[r, k] = cache_type(q[r, k] * s[r]), one rounding of the exact product;
+ * out [rows, head_dim] 16-byte aligned, shape rules of kv_quantize_int8. */
+Q4_API q4_status kv_dequant_int8(const int8_t* codes, const void* scales, q4_dtype dtype,
+                                 int64_t rows, int64_t head_dim, void* out, q4_stream stream);
+
+/* INT4 ("压缩算法" section 7.4.1.2, quantize_kv_cache_int4): the symmetric
+ * group quantizer of q4_quantize_pack (s = fp16(amax / 7), codes in [-8, 7],
+ * two codes per byte, even element in the low nibble) over groups of
+ * group_size values along head_dim.
+ *   packed  [rows, head_dim / 2], 4-byte aligned (written)
+ *   scales  [rows, head_dim / group_size] fp16, 2-byte aligned (written)
+ *   head_dim a multiple of 8; group_size even and dividing head_dim */
+Q4_API q4_status kv_quantize_int4(const void* kv, q4_dtype dtype, int64_t rows, int64_t head_dim,
+                                  int32_t group_size, uint8_t* packed, void* scales,
+                                  q4_stream stream);
+
+/* The dequantization s * q of kv_quantize_int4's output as out_dtype (the
+ * rules of q4_dequant; packed 16-byte aligned). */
+Q4_API q4_status kv_dequant_int4(const uint8_t* packed, const void* scales, int64_t rows,
+                                 int64_t head_dim, int32_t group_size, void* out,
+                                 q4_dtype out_dtype, q4_stream stream);
+
 /*
  * Waits for `stream`, then reports the first device-side error recorded
  * since the previous call (Q4_ERR_TIMEOUT when a kernel's bounded wait ran

@@ -7,7 +7,10 @@ device memory (outputs are allocated here when not given) and the stream
 if ``libq4.so`` cannot be loaded every call raises ``Q4LibraryError``.
 
 Names follow the C ABI: ``q4_quantize_pack``, ``q4_dequant``, ``q4_gemv``,
-``q4_gemm_skinny``, ``bf16_gemv_ref_bw``, ``q4_sync_status``.
+``q4_gemm_skinny``, ``bf16_gemv_ref_bw``, ``q4_sync_status``, the per-channel
+INT8 weight calls ``q8_quantize_per_channel``, ``q8_dequant``, ``q8_gemv`` and
+the KV-cache calls ``kv_quantize_int8``, ``kv_dequant_int8``,
+``kv_quantize_int4``, ``kv_dequant_int4``.
 """
 from __future__ import annotations
 
@@ -37,7 +40,8 @@ ABI_SYMBOLS = (
     "q4_quantize_pack", "q4_dequant", "q4_gemv", "q4_gemm_skinny", "bf16_gemv_ref_bw",
     "q4_sync_status", "q4_status_string", "q4_version", "q4_selftest_wait_timeout",
     "q4_workspace_bytes", "q4_gemv_noalloc", "q4_quantize_pack_clip", "q4_quantize_pack_perm",
-    "q4_permute_activations",
+    "q4_permute_activations", "q8_quantize_per_channel", "q8_dequant", "q8_workspace_bytes",
+    "q8_gemv", "kv_quantize_int8", "kv_dequant_int8", "kv_quantize_int4", "kv_dequant_int4",
 )
 
 
@@ -94,10 +98,21 @@ def load_library(path: str = LIB_PATH):
     lib.bf16_gemv_ref_bw.argtypes = [P, I64, I64, P, I64, P, P]
     lib.q4_sync_status.argtypes = [P]
     lib.q4_selftest_wait_timeout.argtypes = [I64, P]
+    lib.q8_quantize_per_channel.argtypes = [P, S, I64, I64, P, P, P]
+    lib.q8_dequant.argtypes = [P, P, I64, I64, P, S, P]
+    lib.q8_workspace_bytes.argtypes = [I64, I64, I64]
+    lib.q8_workspace_bytes.restype = ctypes.c_size_t
+    lib.q8_gemv.argtypes = [P, P, I64, I64, P, S, I64, P, S, P, ctypes.c_size_t, P]
+    lib.kv_quantize_int8.argtypes = [P, S, I64, I64, P, P, P]
+    lib.kv_dequant_int8.argtypes = [P, P, S, I64, I64, P, P]
+    lib.kv_quantize_int4.argtypes = [P, S, I64, I64, I32, P, P, P]
+    lib.kv_dequant_int4.argtypes = [P, P, I64, I64, I32, P, S, P]
     for f in ("q4_quantize_pack", "q4_quantize_pack_clip", "q4_quantize_pack_perm",
               "q4_permute_activations", "q4_dequant", "q4_gemv",
               "q4_gemm_skinny", "q4_gemv_noalloc",
-              "bf16_gemv_ref_bw", "q4_sync_status", "q4_selftest_wait_timeout"):
+              "bf16_gemv_ref_bw", "q4_sync_status", "q4_selftest_wait_timeout",
+              "q8_quantize_per_channel", "q8_dequant", "q8_gemv", "kv_quantize_int8",
+              "kv_dequant_int8", "kv_quantize_int4", "kv_dequant_int4"):
         getattr(lib, f).restype = S
     lib.q4_status_string.argtypes = [S]
     lib.q4_status_string.restype = ctypes.c_char_p
@@ -272,6 +287,12 @@ def workspace_for(w: Q4Weight, B: int, device) -> torch.Tensor:
     demand; every completed call leaves it zero-filled.  Calls that may
     overlap on the GPU (different streams) must pass their own buffers."""
     need = int(load_library().q4_workspace_bytes(w.out, w.in_features, B, w.group_size))
+    return _shared_workspace(need, device)
+
+
+def _shared_workspace(need: int, device) -> torch.Tensor:
+    """The per-device zero-filled workspace, grown to at least ``need`` bytes
+    (q4 and q8 products share its layout)."""
     dev = torch.device(device)
     key = dev.index if dev.index is not None else torch.cuda.current_device()
     buf = _workspaces.get(key)
@@ -352,3 +373,137 @@ def q4_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
     """Launch a kernel whose bounded wait can never be satisfied; returns the
     launch status (the timeout is then reported by q4_sync_status)."""
     return load_library().q4_selftest_wait_timeout(int(limit_ns), _stream(stream))
+
+
+# ------------------------------------------------ per-channel INT8 weights
+
+@dataclass
+class Q8Weight:
+    """Per-output-channel INT8 weight: codes [out, in] int8, fp32 scales [out]."""
+    qweight: torch.Tensor
+    scales: torch.Tensor
+    out: int
+    in_features: int
+
+    @property
+    def nbytes(self) -> int:
+        return self.qweight.numel() + self.scales.numel() * 4
+
+
+def q8_quantize_per_channel(W: torch.Tensor, qweight: torch.Tensor | None = None,
+                            scales: torch.Tensor | None = None, stream=None) -> Q8Weight:
+    """s[r] = max(amax_r, 1e-6) / 127, q = clamp(rne(W / s), -127, 127)."""
+    lib = load_library()
+    if W.dim() != 2 or W.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("W must be a 2-D fp16 or bf16 tensor")
+    out, inn = W.shape
+    if qweight is None:
+        qweight = torch.empty(out, inn, dtype=torch.int8, device=W.device)
+    if scales is None:
+        scales = torch.empty(out, dtype=torch.float32, device=W.device)
+    st = lib.q8_quantize_per_channel(_ptr(W), _DT[W.dtype], out, inn, _ptr(qweight), _ptr(scales),
+                                     _stream(stream))
+    _check(st, "q8_quantize_per_channel")
+    return Q8Weight(qweight, scales, out, inn)
+
+
+def q8_dequant(w: Q8Weight, out_dtype=torch.float32, W_hat: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    lib = load_library()
+    if W_hat is None:
+        W_hat = torch.empty(w.out, w.in_features, dtype=out_dtype, device=w.qweight.device)
+    st = lib.q8_dequant(_ptr(w.qweight), _ptr(w.scales), w.out, w.in_features, _ptr(W_hat),
+                        _DT[W_hat.dtype], _stream(stream))
+    _check(st, "q8_dequant")
+    return W_hat
+
+
+def q8_gemv(w: Q8Weight, x: torch.Tensor, y: torch.Tensor | None = None, y_dtype=None,
+            workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = x (q * s)^T for B <= 8 (x [B, in] bf16/fp16; y [B, out] x.dtype or fp32)."""
+    lib = load_library()
+    if x.dim() != 2:
+        raise ValueError("x must be [B, in]")
+    B = x.shape[0]
+    if y is None:
+        y = torch.empty(B, w.out, dtype=y_dtype or x.dtype, device=x.device)
+    if workspace is None:
+        workspace = _shared_workspace(int(lib.q8_workspace_bytes(w.out, w.in_features, B)),
+                                      x.device)
+    st = lib.q8_gemv(_ptr(w.qweight), _ptr(w.scales), w.out, w.in_features, _ptr(x), _DT[x.dtype],
+                     B, _ptr(y), _DT[y.dtype], _ptr(workspace),
+                     workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "q8_gemv")
+    return y
+
+
+# ------------------------------------------------------------- KV cache
+
+def _kv_rows(kv: torch.Tensor):
+    if kv.dim() < 1 or kv.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("kv must be an fp16 or bf16 tensor [..., head_dim]")
+    d = kv.shape[-1]
+    return kv.numel() // d if d else 0, d
+
+
+def kv_quantize_int8(kv: torch.Tensor, codes: torch.Tensor | None = None,
+                     scales: torch.Tensor | None = None, stream=None):
+    """INT8 along head_dim, one scale per row in the cache's dtype.
+    Returns (codes int8 kv.shape, scales kv.shape[:-1])."""
+    lib = load_library()
+    rows, d = _kv_rows(kv)
+    if codes is None:
+        codes = torch.empty(kv.shape, dtype=torch.int8, device=kv.device)
+    if scales is None:
+        scales = torch.empty(kv.shape[:-1], dtype=kv.dtype, device=kv.device)
+    st = lib.kv_quantize_int8(_ptr(kv), _DT[kv.dtype], rows, d, _ptr(codes), _ptr(scales),
+                              _stream(stream))
+    _check(st, "kv_quantize_int8")
+    return codes, scales
+
+
+def kv_dequant_int8(codes: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """cache_type(q * s), in the dtype of ``scales``."""
+    lib = load_library()
+    d = codes.shape[-1]
+    rows = codes.numel() // d if d else 0
+    if out is None:
+        out = torch.empty(codes.shape, dtype=scales.dtype, device=codes.device)
+    st = lib.kv_dequant_int8(_ptr(codes), _ptr(scales), _DT[scales.dtype], rows, d, _ptr(out),
+                             _stream(stream))
+    _check(st, "kv_dequant_int8")
+    return out
+
+
+def kv_quantize_int4(kv: torch.Tensor, group_size: int = 128, packed: torch.Tensor | None = None,
+                     scales: torch.Tensor | None = None, stream=None):
+    """INT4 groups of group_size along head_dim (fp16 scales, codes in
+    [-8, 7], two per byte).  Returns (packed uint8 [..., d/2], scales fp16
+    [..., d/group_size])."""
+    lib = load_library()
+    rows, d = _kv_rows(kv)
+    lead = tuple(kv.shape[:-1])
+    if packed is None:
+        packed = torch.empty(lead + (d // 2,), dtype=torch.uint8, device=kv.device)
+    if scales is None:
+        G = d // group_size if group_size > 0 else 0
+        scales = torch.empty(lead + (G,), dtype=torch.float16, device=kv.device)
+    st = lib.kv_quantize_int4(_ptr(kv), _DT[kv.dtype], rows, d, group_size, _ptr(packed),
+                              _ptr(scales), _stream(stream))
+    _check(st, "kv_quantize_int4")
+    return packed, scales
+
+
+def kv_dequant_int4(packed: torch.Tensor, scales: torch.Tensor, group_size: int = 128,
+                    out_dtype=torch.float16, out: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    lib = load_library()
+    d = packed.shape[-1] * 2
+    rows = packed.numel() * 2 // d if d else 0
+    if out is None:
+        out = torch.empty(tuple(packed.shape[:-1]) + (d,), dtype=out_dtype, device=packed.device)
+    st = lib.kv_dequant_int4(_ptr(packed), _ptr(scales), rows, d, group_size, _ptr(out),
+                             _DT[out.dtype], _stream(stream))
+    _check(st, "kv_dequant_int4")
+    return out

@@ -1,6 +1,7 @@
 // q4_api.cu -- the C ABI of include/q4.h: argument validation, launch
 // planning, TMA descriptor encoding and kernel launches.  All kernels live in
-// this translation unit (q4_quant.cuh, q4_gemv.cuh, q4_skinny.cuh).
+// this translation unit (q4_quant.cuh, q4_gemv.cuh, q4_gemv_sk.cuh,
+// q4_skinny_tc.cuh, q8_gemv.cuh, q8_quant.cuh).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -17,6 +18,8 @@
 #include "q4_gemv_sk.cuh"
 #include "q4_quant.cuh"
 #include "q4_skinny_tc.cuh"
+#include "q8_gemv.cuh"
+#include "q8_quant.cuh"
 
 namespace {
 
@@ -292,13 +295,14 @@ struct SkPlan {
     size_t ws_part_bytes, ws_bytes;
 };
 
-// Stream-K plan over row tiles of `rt` rows and 256-code chunks: at least
-// `min_iters` iterations per CTA (tiny problems use fewer SMs rather than
-// paying a fixup for every chunk), at most `pmax` CTAs; each CTA has two
-// partial slots of rt x `cols` fp32.
-SkPlan stream_k_plan(int64_t out, int64_t in, int rt, int64_t pmax, int min_iters, int cols) {
+// Stream-K plan over row tiles of `rt` rows and chunks of `chunk_codes`
+// codes of K: at least `min_iters` iterations per CTA (tiny problems use
+// fewer SMs rather than paying a fixup for every chunk), at most `pmax` CTAs;
+// each CTA has two partial slots of rt x `cols` fp32.
+SkPlan stream_k_plan(int64_t out, int64_t in, int rt, int64_t pmax, int min_iters, int cols,
+                     int chunk_codes = kChunkCodes) {
     SkPlan p{};
-    p.nchunks = static_cast<int>((in + kChunkCodes - 1) / kChunkCodes);
+    p.nchunks = static_cast<int>((in + chunk_codes - 1) / chunk_codes);
     p.row_tiles = (out + rt - 1) / rt;
     p.T = p.row_tiles * p.nchunks;
     p.P = std::min<int64_t>(std::max<int64_t>(1, p.T / min_iters), pmax);
@@ -400,6 +404,49 @@ q4_status dispatch_gemv(const q4_weight* w, const void* x, int64_t B, void* y, i
                              : run_gemv<BF16, 128, false>(w, x, B, y, ydt, ws, wsb, st);
         default: return Q4_ERR_UNSUPPORTED;
     }
+}
+
+// ------------------------------------------- W8A16 (per-channel INT8)
+constexpr int kQ8CW = 8;
+constexpr int kQ8RT = kQ8CW * 16;
+
+SkPlan q8_plan(int64_t out, int64_t in, int sms) {
+    return stream_k_plan(out, in, kQ8RT, static_cast<int64_t>(kSkCtasPerSm) * sms, kSkMinIters, 8,
+                         kQ8ChunkCodes);
+}
+
+template <bool BF16>
+q4_status run_q8_gemv(const int8_t* qweight, const float* scales, int64_t out, int64_t in,
+                      const void* x, int64_t B, void* y, int ydt, void* ws, size_t ws_bytes,
+                      cudaStream_t st) {
+    const int dev = current_device();
+    const SkPlan p = q8_plan(out, in, sm_count(dev));
+    if (!ws || ws_bytes < p.ws_bytes) return Q4_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return Q4_ERR_ALIGNMENT;
+    // deepest ring that still lets two CTAs share an SM
+    const size_t per_sm = 228 * 1024;
+    int stages = kQ8MaxStages;
+    Q8Geom geo = q8_geom(kQ8RT, stages);
+    while (stages > 2 && kSkCtasPerSm * (geo.total + 1024) > per_sm) geo = q8_geom(kQ8RT, --stages);
+    CUtensorMap tmap_w, tmap_x;
+    if (!make_tmap_2d(&tmap_w, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                      static_cast<uint64_t>(out), static_cast<uint64_t>(in), kQ8RT, kChunkBytes))
+        return Q4_ERR_CUDA;
+    if (!make_tmap_2d(&tmap_x, x,
+                      BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                      static_cast<uint64_t>(B), static_cast<uint64_t>(in),
+                      static_cast<uint32_t>(B), 64))
+        return Q4_ERR_CUDA;
+    auto kernel = q8_gemv_sk_kernel<BF16, kQ8CW>;
+    if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), false)) return Q4_ERR_CUDA;
+    unsigned* status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
+        return Q4_ERR_CUDA;
+    unsigned* ws_count = reinterpret_cast<unsigned*>(ws);
+    float* ws_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kWsCounterBytes);
+    return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3((kQ8CW + 1) * 32), geo.total,
+                     1, true, st, tmap_w, tmap_x, scales, stages, static_cast<int>(B), out, in,
+                     p.nchunks, p.T, y, ydt, ws_part, ws_count, status);
 }
 
 template <bool BF16, int GS, int NT>
@@ -798,6 +845,176 @@ q4_status bf16_gemv_ref_bw(const void* W, int64_t out, int64_t in, const void* x
     return launch_cluster(kernel, grid, dim3((kGemvCW + 1) * 32), geo.total, p.S, st, tmap,
                           reinterpret_cast<const uint16_t*>(x), static_cast<int>(B), out, in,
                           p.cps, nchunks, y, status);
+}
+
+// ------------------------------------------------- per-channel INT8 weights
+
+q4_status q8_quantize_per_channel(const void* W, q4_dtype w_dtype, int64_t out, int64_t in,
+                                  int8_t* qweight, float* scales, q4_stream stream) {
+    if (w_dtype != Q4_F16 && w_dtype != Q4_BF16) {
+        return valid_dtype(w_dtype) ? Q4_ERR_UNSUPPORTED : Q4_ERR_INVALID_ARG;
+    }
+    if (out < 0 || in <= 0 || (in % 16) != 0) return Q4_ERR_SHAPE;
+    if (out == 0) return Q4_OK;
+    if (!W || !qweight || !scales) return Q4_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(qweight, 16) || !aligned(scales, 4)) return Q4_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int sms = sm_count(current_device());
+    const int blocks = static_cast<int>(out < 16LL * sms ? out : 16LL * sms);
+    if (w_dtype == Q4_BF16)
+        q8_quantize_rows_kernel<true><<<blocks, 256, 0, st>>>(W, out, in, qweight, scales);
+    else
+        q8_quantize_rows_kernel<false><<<blocks, 256, 0, st>>>(W, out, in, qweight, scales);
+    return launch_status(cudaSuccess);
+}
+
+q4_status q8_dequant(const int8_t* qweight, const float* scales, int64_t out, int64_t in,
+                     void* W_hat, q4_dtype out_dtype, q4_stream stream) {
+    if (!valid_dtype(out_dtype)) return Q4_ERR_INVALID_ARG;
+    if (out < 0 || in <= 0 || (in % 16) != 0) return Q4_ERR_SHAPE;
+    if (out == 0) return Q4_OK;
+    if (!qweight || !scales || !W_hat) return Q4_ERR_INVALID_ARG;
+    if (!aligned(qweight, 16) || !aligned(scales, 4) || !aligned(W_hat, 16))
+        return Q4_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int sms = sm_count(current_device());
+    const int64_t nvec = out * in / 8;
+    const int64_t want = (nvec + 255) / 256;
+    const int blocks = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
+    if (out_dtype == Q4_F32)
+        q8_dequant_kernel<float><<<blocks, 256, 0, st>>>(qweight, scales, nvec, in,
+                                                         reinterpret_cast<float*>(W_hat));
+    else if (out_dtype == Q4_F16)
+        q8_dequant_kernel<__half><<<blocks, 256, 0, st>>>(qweight, scales, nvec, in,
+                                                          reinterpret_cast<__half*>(W_hat));
+    else
+        q8_dequant_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+            qweight, scales, nvec, in, reinterpret_cast<__nv_bfloat16*>(W_hat));
+    return launch_status(cudaSuccess);
+}
+
+size_t q8_workspace_bytes(int64_t out, int64_t in, int64_t B) {
+    if (out <= 0 || in <= 0 || B < 1 || B > 8) return 0;
+    return q8_plan(out, in, sm_count(current_device())).ws_bytes;
+}
+
+q4_status q8_gemv(const int8_t* qweight, const float* scales, int64_t out, int64_t in,
+                  const void* x, q4_dtype x_dtype, int64_t B, void* y, q4_dtype y_dtype,
+                  void* workspace, size_t workspace_bytes, q4_stream stream) {
+    if (!valid_dtype(x_dtype) || !valid_dtype(y_dtype)) return Q4_ERR_INVALID_ARG;
+    if (x_dtype == Q4_F32) return Q4_ERR_UNSUPPORTED;
+    if (y_dtype != x_dtype && y_dtype != Q4_F32) return Q4_ERR_UNSUPPORTED;
+    if (B < 1 || B > 8) return Q4_ERR_SHAPE;
+    if (out < 0 || in <= 0 || (in % 16) != 0) return Q4_ERR_SHAPE;
+    if (in > (int64_t(1) << 30) || out > int64_t(65535) * kQ8RT) return Q4_ERR_SHAPE;
+    if (out == 0) return Q4_OK;
+    if (!qweight || !scales || !x || !y) return Q4_ERR_INVALID_ARG;
+    if (!aligned(qweight, 16) || !aligned(scales, 4) || !aligned(x, 16) || !aligned(y, 16))
+        return Q4_ERR_ALIGNMENT;
+    if (!workspace) return Q4_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int ydt = y_dtype == Q4_F32 ? 2 : (y_dtype == Q4_BF16 ? 1 : 0);
+    return x_dtype == Q4_BF16 ? run_q8_gemv<true>(qweight, scales, out, in, x, B, y, ydt, workspace,
+                                                  workspace_bytes, st)
+                              : run_q8_gemv<false>(qweight, scales, out, in, x, B, y, ydt,
+                                                   workspace, workspace_bytes, st);
+}
+
+// ------------------------------------------------------------- KV cache
+
+q4_status kv_quantize_int8(const void* kv, q4_dtype dtype, int64_t rows, int64_t head_dim,
+                           int8_t* codes, void* scales, q4_stream stream) {
+    if (dtype != Q4_F16 && dtype != Q4_BF16) {
+        return valid_dtype(dtype) ? Q4_ERR_UNSUPPORTED : Q4_ERR_INVALID_ARG;
+    }
+    if (rows < 0 || head_dim < 8 || head_dim > 512 || (head_dim % 8) != 0) return Q4_ERR_SHAPE;
+    if (rows == 0) return Q4_OK;
+    if (!kv || !codes || !scales) return Q4_ERR_INVALID_ARG;
+    if (!aligned(kv, 16) || !aligned(codes, 16) || !aligned(scales, 2)) return Q4_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int sms = sm_count(current_device());
+    const int d = static_cast<int>(head_dim);
+    const int V = d / 8;
+    int ts = 1;
+    while (ts * 2 < V) ts *= 2;  // smallest power of two with 2 * ts >= V
+    const int64_t rpw = 32 / ts;
+    const int64_t warps = (rows + rpw - 1) / rpw;
+    const int64_t want = (warps + 7) / 8;
+    const int blocks = static_cast<int>(want < 16LL * sms ? want : 16LL * sms);
+    const uint16_t* in = reinterpret_cast<const uint16_t*>(kv);
+    uint16_t* sc = reinterpret_cast<uint16_t*>(scales);
+    const bool bf = dtype == Q4_BF16;
+    switch (ts) {
+#define Q4_KVCASE(TSV)                                                                          \
+    case TSV:                                                                                   \
+        if (bf)                                                                                 \
+            kv_quantize_int8_kernel<true, TSV><<<blocks, 256, 0, st>>>(in, rows, d, codes, sc); \
+        else                                                                                    \
+            kv_quantize_int8_kernel<false, TSV><<<blocks, 256, 0, st>>>(in, rows, d, codes, sc); \
+        break;
+        Q4_KVCASE(1) Q4_KVCASE(2) Q4_KVCASE(4) Q4_KVCASE(8) Q4_KVCASE(16) Q4_KVCASE(32)
+#undef Q4_KVCASE
+        default: return Q4_ERR_SHAPE;
+    }
+    return launch_status(cudaSuccess);
+}
+
+q4_status kv_dequant_int8(const int8_t* codes, const void* scales, q4_dtype dtype, int64_t rows,
+                          int64_t head_dim, void* out, q4_stream stream) {
+    if (dtype != Q4_F16 && dtype != Q4_BF16) {
+        return valid_dtype(dtype) ? Q4_ERR_UNSUPPORTED : Q4_ERR_INVALID_ARG;
+    }
+    if (rows < 0 || head_dim < 8 || head_dim > 512 || (head_dim % 8) != 0) return Q4_ERR_SHAPE;
+    if (rows == 0) return Q4_OK;
+    if (!codes || !scales || !out) return Q4_ERR_INVALID_ARG;
+    if (!aligned(codes, 16) || !aligned(scales, 2) || !aligned(out, 16)) return Q4_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int sms = sm_count(current_device());
+    const int64_t nvec = rows * head_dim / 8;
+    const int64_t want = (nvec + 255) / 256;
+    const int blocks = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
+    const uint16_t* sc = reinterpret_cast<const uint16_t*>(scales);
+    uint16_t* o = reinterpret_cast<uint16_t*>(out);
+    if (dtype == Q4_BF16)
+        kv_dequant_int8_kernel<true><<<blocks, 256, 0, st>>>(codes, sc, nvec,
+                                                             static_cast<int>(head_dim), o);
+    else
+        kv_dequant_int8_kernel<false><<<blocks, 256, 0, st>>>(codes, sc, nvec,
+                                                              static_cast<int>(head_dim), o);
+    return launch_status(cudaSuccess);
+}
+
+q4_status kv_quantize_int4(const void* kv, q4_dtype dtype, int64_t rows, int64_t head_dim,
+                           int32_t group_size, uint8_t* packed, void* scales, q4_stream stream) {
+    if (dtype != Q4_F16 && dtype != Q4_BF16) {
+        return valid_dtype(dtype) ? Q4_ERR_UNSUPPORTED : Q4_ERR_INVALID_ARG;
+    }
+    if (rows < 0 || head_dim <= 0 || (head_dim % 8) != 0 || group_size <= 0) return Q4_ERR_SHAPE;
+    if ((group_size & 1) || (head_dim % group_size) != 0) return Q4_ERR_SHAPE;
+    if (rows == 0) return Q4_OK;
+    if (!kv || !packed || !scales) return Q4_ERR_INVALID_ARG;
+    if (!aligned(kv, 16) || !aligned(packed, 4) || !aligned(scales, 2)) return Q4_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    __half* s = reinterpret_cast<__half*>(scales);
+    return dtype == Q4_BF16
+               ? run_quantize<true, true>(kv, rows, head_dim, group_size, packed, s, nullptr, st)
+               : run_quantize<true, false>(kv, rows, head_dim, group_size, packed, s, nullptr, st);
+}
+
+q4_status kv_dequant_int4(const uint8_t* packed, const void* scales, int64_t rows,
+                          int64_t head_dim, int32_t group_size, void* out, q4_dtype out_dtype,
+                          q4_stream stream) {
+    if (rows < 0 || head_dim <= 0) return Q4_ERR_SHAPE;
+    q4_weight w{};
+    w.qweight = packed;
+    w.scales = scales;
+    w.zeros = nullptr;
+    w.out = rows;
+    w.in = head_dim;
+    w.group_size = group_size;
+    w.bits = 4;
+    w.symmetric = 1;
+    return q4_dequant(&w, out, out_dtype, stream);
 }
 
 q4_status q4_selftest_wait_timeout(int64_t limit_ns, q4_stream stream) {

@@ -105,3 +105,24 @@ def llama3_8b_layer_seeds(layer: int) -> dict:
 def llama3_70b_stack_seed(layer: int, idx: int) -> int:
     """Seed of linear ``idx`` (0..6 in LLAMA3_70B order) of layer ``layer``."""
     return 1000 * layer + idx
+
+
+# Llama-3-70B KV cache geometry: 8 KV heads of head_dim 128 per layer
+# ("LLM 后训练量化深度实战" (ybb.press) section 七, the KV bytes per token).
+LLAMA3_70B_KV_HEADS = 8
+LLAMA3_70B_HEAD_DIM = 128
+
+
+def kv_cache(batch: int, heads: int, seq: int, head_dim: int, seed: int, dtype=torch.float16,
+             n_sink: int = 4, sink_scale: float = 30.0, device="cpu") -> torch.Tensor:
+    """A synthetic K or V cache [batch, heads, seq, head_dim]: N(0, 1) values
+    times a per-head magnitude drawn log-uniformly from [0.1, 10], with the
+    first ``n_sink`` tokens of every head scaled by ``sink_scale`` (the
+    large-magnitude attention-sink tokens of ybb.press section 七)."""
+    g = _gen(seed, device)
+    x = torch.randn(batch, heads, seq, head_dim, generator=g, device=device, dtype=torch.float32)
+    mag = torch.exp(torch.empty(1, heads, 1, 1, device=device).uniform_(-2.3026, 2.3026, generator=g))
+    x = x * mag
+    if n_sink:
+        x[:, :, :n_sink, :] *= sink_scale
+    return x.to(dtype)

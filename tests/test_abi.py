@@ -212,3 +212,62 @@ def test_act_order_validation(lib):
     assert p(None, q4.Q4_BF16, 2, 128, A16, A16, None) == q4.Q4_ERR_INVALID_ARG
     assert p(A16, q4.Q4_BF16, 2, 128, A16, A2, None) == q4.Q4_ERR_ALIGNMENT
     assert p(A16, q4.Q4_BF16, 0, 128, A16, A16, None) == q4.Q4_OK
+
+
+def test_q8_weight_validation(lib):
+    qz = lib.q8_quantize_per_channel
+    assert qz(A16, q4.Q4_F32, 8, 256, A16, A16, None) == q4.Q4_ERR_UNSUPPORTED
+    assert qz(A16, 7, 8, 256, A16, A16, None) == q4.Q4_ERR_INVALID_ARG
+    assert qz(A16, q4.Q4_BF16, 8, 200, A16, A16, None) == q4.Q4_ERR_SHAPE   # in % 16
+    assert qz(A16, q4.Q4_BF16, -1, 256, A16, A16, None) == q4.Q4_ERR_SHAPE
+    assert qz(A16, q4.Q4_BF16, 0, 256, A16, A16, None) == q4.Q4_OK
+    assert qz(None, q4.Q4_BF16, 8, 256, A16, A16, None) == q4.Q4_ERR_INVALID_ARG
+    assert qz(A16, q4.Q4_BF16, 8, 256, A2, A16, None) == q4.Q4_ERR_ALIGNMENT
+    assert qz(A16, q4.Q4_BF16, 8, 256, A16, A2, None) == q4.Q4_ERR_ALIGNMENT
+    dq = lib.q8_dequant
+    assert dq(A16, A16, 8, 256, A16, 9, None) == q4.Q4_ERR_INVALID_ARG
+    assert dq(A16, A16, 8, 24, A16, q4.Q4_F32, None) == q4.Q4_ERR_SHAPE
+    assert dq(A16, A16, 0, 256, A16, q4.Q4_F32, None) == q4.Q4_OK
+    assert dq(A16, A16, 8, 256, A2, q4.Q4_F32, None) == q4.Q4_ERR_ALIGNMENT
+    g = lib.q8_gemv
+    ok = dict(q=A16, s=A16, out=64, inn=256, x=A16, xdt=q4.Q4_BF16, B=1, y=A16, ydt=q4.Q4_BF16,
+              ws=None, wsb=0)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return g(a["q"], a["s"], a["out"], a["inn"], a["x"], a["xdt"], a["B"], a["y"], a["ydt"],
+                 a["ws"], a["wsb"], None)
+
+    assert call() == q4.Q4_ERR_WORKSPACE
+    assert call(xdt=q4.Q4_F32) == q4.Q4_ERR_UNSUPPORTED
+    assert call(ydt=q4.Q4_F16) == q4.Q4_ERR_UNSUPPORTED   # bf16 x, fp16 y
+    assert call(B=0) == q4.Q4_ERR_SHAPE and call(B=9) == q4.Q4_ERR_SHAPE
+    assert call(inn=120) == q4.Q4_ERR_SHAPE
+    assert call(out=0) == q4.Q4_OK
+    assert call(x=None) == q4.Q4_ERR_INVALID_ARG
+    assert call(x=A2) == q4.Q4_ERR_ALIGNMENT and call(s=A2) == q4.Q4_ERR_ALIGNMENT
+    assert lib.q8_workspace_bytes(64, 256, 9) == 0 and lib.q8_workspace_bytes(0, 256, 1) == 0
+
+
+def test_kv_cache_validation(lib):
+    k8 = lib.kv_quantize_int8
+    assert k8(A16, q4.Q4_F32, 4, 128, A16, A16, None) == q4.Q4_ERR_UNSUPPORTED
+    assert k8(A16, q4.Q4_F16, 4, 100, A16, A16, None) == q4.Q4_ERR_SHAPE    # head_dim % 8
+    assert k8(A16, q4.Q4_F16, 4, 520, A16, A16, None) == q4.Q4_ERR_SHAPE    # > 512
+    assert k8(A16, q4.Q4_F16, 0, 128, A16, A16, None) == q4.Q4_OK
+    assert k8(A16, q4.Q4_F16, 4, 128, None, A16, None) == q4.Q4_ERR_INVALID_ARG
+    assert k8(A2, q4.Q4_F16, 4, 128, A16, A16, None) == q4.Q4_ERR_ALIGNMENT
+    d8 = lib.kv_dequant_int8
+    assert d8(A16, A16, q4.Q4_BF16, 4, 128, A2, None) == q4.Q4_ERR_ALIGNMENT
+    assert d8(A16, A16, q4.Q4_BF16, 4, 4, A16, None) == q4.Q4_ERR_SHAPE
+    assert d8(A16, A16, q4.Q4_BF16, 0, 128, A16, None) == q4.Q4_OK
+    k4 = lib.kv_quantize_int4
+    assert k4(A16, q4.Q4_BF16, 4, 128, 96, A16, A16, None) == q4.Q4_ERR_SHAPE   # 96 does not divide
+    assert k4(A16, q4.Q4_BF16, 4, 128, 127, A16, A16, None) == q4.Q4_ERR_SHAPE  # odd group
+    assert k4(A16, q4.Q4_BF16, 0, 128, 128, A16, A16, None) == q4.Q4_OK
+    assert k4(A16, q4.Q4_BF16, 4, 128, 128, A2, A16, None) == q4.Q4_ERR_ALIGNMENT
+    d4 = lib.kv_dequant_int4
+    assert d4(A16, A16, 4, 128, 128, None, q4.Q4_F16, None) == q4.Q4_ERR_INVALID_ARG
+    assert d4(A16, A16, 4, 128, 96, A16, q4.Q4_F16, None) == q4.Q4_ERR_SHAPE
+    assert d4(A16, A16, 0, 128, 128, A16, q4.Q4_F16, None) == q4.Q4_OK
