@@ -676,13 +676,65 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_op(args):
+    """One operation of the path alone, for profiling and spot timing:
+    ``w8a16-70b`` = q8_gemv on the Llama-3-70B down_proj (8192 x 28672, batch
+    --batch, two weight copies rotating); ``kv8-70b-32k`` = kv_quantize_int8
+    of one layer's K cache at 32768 tokens ([1, 8, 32768, 128] bf16, four
+    caches rotating).  Prints one JSON line (CUDA-event time per call)."""
+    import torch
+    sys.path.insert(0, ROOT)
+    import post_weight_quantization_group_b200 as q4
+    from post_weight_quantization_group_b200 import workloads as wl
+    q4.load_library()
+    device = torch.device("cuda:0")
+    stream = torch.cuda.current_stream()
+    if args.workload == "w8a16-70b":
+        out, inn = wl.LLAMA3_70B["down_proj"]
+        B = args.batch
+        ws = []
+        for i in range(2):
+            W = wl.normal_weight(out, inn, 60 + i, device=device).to(torch.bfloat16)
+            ws.append(q4.q8_quantize_per_channel(W))
+            del W
+        torch.cuda.empty_cache()
+        x = wl.activations(B, inn, 61, device=device)
+        y = torch.empty(B, out, dtype=torch.bfloat16, device=device)
+        wsp = q4._shared_workspace(int(q4.load_library().q8_workspace_bytes(out, inn, B)), device)
+        it = iter(range(1 << 30))
+        fn = lambda: q4.q8_gemv(ws[next(it) % 2], x, y=y, workspace=wsp)
+        nbytes = out * inn + out * 4 + B * inn * 2 + B * out * 2
+        name, cfg = "W8A16 per-channel INT8 GEMV", {"workload": f"Llama-3-70B down_proj {out}x{inn}", "batch": B}
+    else:
+        shape = (1, wl.LLAMA3_70B_KV_HEADS, 32768, wl.LLAMA3_70B_HEAD_DIM)
+        caches = [wl.kv_cache(*shape, seed=70 + i, dtype=torch.bfloat16, device=device) for i in range(4)]
+        c8 = [torch.empty(shape, dtype=torch.int8, device=device) for _ in range(4)]
+        s8 = [torch.empty(shape[:-1], dtype=torch.bfloat16, device=device) for _ in range(4)]
+        it = iter(range(1 << 30))
+
+        def fn():
+            i = next(it) % 4
+            q4.kv_quantize_int8(caches[i], c8[i], s8[i])
+        n = caches[0].numel()
+        nbytes = 3 * n + 2 * (n // shape[-1])
+        name, cfg = "INT8 KV-cache quantization", {"workload": "Llama-3-70B K cache [1,8,32768,128] bf16"}
+    ms = time_region(torch, fn, args.steps, args.warmup, stream) / args.steps
+    st = q4.q4_sync_status()
+    assert st == q4.Q4_OK, q4.status_string(st)
+    print(json.dumps({"metric": name, "value": round(nbytes / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                      "us_per_call": round(ms * 1e3, 2), "steps": args.steps, "warmup": args.warmup,
+                      "config": cfg, "timing": "CUDA events on the launching stream, eager launches"}),
+          flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llama3-8b", choices=["llama3-8b", "llama3-70b-stack"])
+    ap.add_argument("--workload", default="llama3-8b",
+                    choices=["llama3-8b", "llama3-70b-stack", "w8a16-70b", "kv8-70b-32k"])
     ap.add_argument("--batch", type=int, default=1, help="batch of the llama3-70b-stack workload")
     ap.add_argument("--layers", type=int, default=32,
                     help="distinct decoder layers per step (32 = the Llama-3-8B depth)")
@@ -697,6 +749,8 @@ def main():
         run_reference(args)
     elif args.workload == "llama3-70b-stack":
         run_stack(args)
+    elif args.workload in ("w8a16-70b", "kv8-70b-32k"):
+        run_op(args)
     else:
         run_ours(args)
 

@@ -70,10 +70,12 @@ __device__ __forceinline__ void load8_perm_f32(const void* base, int64_t r, int6
     }
 }
 
-// clamp(rne(w / s) + z, qmin, qmax) with the same fp32 operations as the
-// definition: IEEE division, round half to even, add z, clamp (NaN -> qmin).
-__device__ __forceinline__ int quant_one(float w, float s, float z, float qmin, float qmax) {
-    float t = rintf(__fdiv_rn(w, s));
+// clamp(rne(w / s) + z, qmin, qmax) with the result of the definition's fp32
+// operations: IEEE division (through rne_quot, r = quot_recip(s)), round half
+// to even, add z, clamp (NaN -> qmin).
+__device__ __forceinline__ int quant_one(float w, float s, float r, float z, float qmin,
+                                         float qmax) {
+    float t = rne_quot(w, s, r);
     t = __fadd_rn(t, z);
     t = fminf(fmaxf(t, qmin), qmax);
     return static_cast<int>(t);
@@ -120,9 +122,10 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const void* __restri
             s32 = __fdiv_rn(a, 7.0f);
             sf = __half2float(__float2half_rn(s32));
             if (sf != 0.f) {
+                const float rf = quot_recip(sf);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const int q = quant_one(v[e], sf, 0.f, -8.f, 7.f);
+                    const int q = quant_one(v[e], sf, rf, 0.f, -8.f, 7.f);
                     packed |= (static_cast<uint32_t>(q) & 0xFu) << (4 * e);
                 }
             }
@@ -141,10 +144,11 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const void* __restri
             s32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
             sf = __half2float(__float2half_rn(s32));
             if (sf != 0.f) {
-                zf = static_cast<float>(quant_one(-mn, sf, 0.f, 0.f, 15.f));
+                const float rf = quot_recip(sf);
+                zf = static_cast<float>(quant_one(-mn, sf, rf, 0.f, 0.f, 15.f));
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const int q = quant_one(v[e], sf, zf, 0.f, 15.f);
+                    const int q = quant_one(v[e], sf, rf, zf, 0.f, 15.f);
                     packed |= (static_cast<uint32_t>(q) & 0xFu) << (4 * e);
                 }
             }
@@ -206,9 +210,10 @@ __global__ void __launch_bounds__(256) quantize_pack_clip_kernel(const void* __r
             const float sf = __half2float(s16);
             uint32_t packed = 0;
             double e = 0.0;
+            const float rf = quot_recip(sf);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                const int q = (sf == 0.f) ? 0 : quant_one(v[k], sf, 0.f, -7.f, 7.f);
+                const int q = (sf == 0.f) ? 0 : quant_one(v[k], sf, rf, 0.f, -7.f, 7.f);
                 packed |= (static_cast<uint32_t>(q) & 0xFu) << (4 * k);
                 const double d = static_cast<double>(v[k]) - static_cast<double>(sf) * q;
                 e += d * d;
@@ -271,16 +276,17 @@ __global__ void __launch_bounds__(256) quantize_pack_generic_kernel(
             s32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
         }
         const float sf = __half2float(__float2half_rn(s32));
-        if (!SYM && sf != 0.f) zf = static_cast<float>(quant_one(-mn, sf, 0.f, 0.f, 15.f));
+        const float rf = quot_recip(sf);
+        if (!SYM && sf != 0.f) zf = static_cast<float>(quant_one(-mn, sf, rf, 0.f, 0.f, 15.f));
         for (int p = lane; p < g / 2; p += 32) {
             int q0 = 0, q1 = 0;
             if (sf != 0.f) {
                 if constexpr (SYM) {
-                    q0 = quant_one(ld(base + 2 * p), sf, 0.f, -8.f, 7.f);
-                    q1 = quant_one(ld(base + 2 * p + 1), sf, 0.f, -8.f, 7.f);
+                    q0 = quant_one(ld(base + 2 * p), sf, rf, 0.f, -8.f, 7.f);
+                    q1 = quant_one(ld(base + 2 * p + 1), sf, rf, 0.f, -8.f, 7.f);
                 } else {
-                    q0 = quant_one(ld(base + 2 * p), sf, zf, 0.f, 15.f);
-                    q1 = quant_one(ld(base + 2 * p + 1), sf, zf, 0.f, 15.f);
+                    q0 = quant_one(ld(base + 2 * p), sf, rf, zf, 0.f, 15.f);
+                    q1 = quant_one(ld(base + 2 * p + 1), sf, rf, zf, 0.f, 15.f);
                 }
             }
             qweight[base / 2 + p] =

@@ -4,7 +4,8 @@
 // Weights ("量化：PTQ、GPTQ、AWQ 与 SmoothQuant" (charles2530.github.io)
 // section 13, per_channel_int8_quant), one scale per row of W [out, in]:
 //   s = max(max_k |w|, 1e-6) / 127,   q = clamp(rne(w / s), -127, 127)
-// in fp32 with IEEE divisions; s is stored as fp32 and w_hat = q * s.
+// in fp32 with the results of IEEE divisions (rne_quot); s is stored as fp32
+// and w_hat = q * s.
 //
 // KV cache ("压缩算法" (cs-knowledge-wiki) section 7.4.1.1,
 // quantize_kv_cache_int8 along the last axis), one scale per row of head_dim
@@ -53,13 +54,14 @@ __global__ void __launch_bounds__(256)
         }
         __syncthreads();
         const float s = s_row;
+        const float rs = quot_recip(s);
         for (int64_t k = static_cast<int64_t>(threadIdx.x) * 8; k < in; k += 256 * 8) {
             float v[8];
             load8_f32<BF16IN>(W, r * in + k, v);
             uint32_t packed[2] = {0u, 0u};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                float t = rintf(__fdiv_rn(v[i], s));
+                float t = rne_quot(v[i], s, rs);
                 t = fminf(fmaxf(t, -127.f), 127.f);  // a NaN quotient becomes -127
                 const uint32_t b = static_cast<uint32_t>(static_cast<int>(t)) & 0xFFu;
                 packed[i >> 2] |= b << (8 * (i & 3));
@@ -161,6 +163,7 @@ __global__ void __launch_bounds__(256)
         for (int off = TS / 2; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
         const uint16_t sbits = cache_bits<BF16>(__fdiv_rn(a, 127.0f));
         const float s = cache_value<BF16>(sbits);
+        const float rs = quot_recip(s);
         if (live && sub == 0) scales[r] = sbits;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -171,7 +174,7 @@ __global__ void __launch_bounds__(256)
             for (int i = 0; i < 8; ++i) {
                 float t = 0.f;
                 if (s != 0.f) {
-                    t = rintf(__fdiv_rn(v[h][i], s));
+                    t = rne_quot(v[h][i], s, rs);
                     t = fminf(fmaxf(t, -128.f), 127.f);
                 }
                 const uint32_t b = static_cast<uint32_t>(static_cast<int>(t)) & 0xFFu;
