@@ -88,6 +88,18 @@ def _load():
     lib.oracle_q8_gemv_rows_f64.argtypes = [P, P, I64, I64, P, I64, P, I64, P]
     lib.oracle_kv_quantize_int8.argtypes = [P, I64, I64, I32, P, P]
     lib.oracle_kv_dequant_int8.argtypes = [P, P, I64, I64, I32, P]
+    lib.oracle_e2m1_to_f32.argtypes = [ctypes.c_uint8]
+    lib.oracle_e2m1_to_f32.restype = ctypes.c_float
+    lib.oracle_f32_to_e2m1.argtypes = [ctypes.c_float]
+    lib.oracle_f32_to_e2m1.restype = ctypes.c_uint8
+    lib.oracle_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_to_f32.restype = ctypes.c_float
+    lib.oracle_f32_to_e4m3_sat.argtypes = [ctypes.c_float]
+    lib.oracle_f32_to_e4m3_sat.restype = ctypes.c_uint8
+    lib.oracle_mxfp4_quantize.argtypes = [P, I64, I64, P, P]
+    lib.oracle_mxfp4_dequant.argtypes = [P, P, I64, I64, P]
+    lib.oracle_nvfp4_quantize.argtypes = [P, I64, I64, P, P, P]
+    lib.oracle_nvfp4_dequant.argtypes = [P, P, ctypes.c_float, I64, I64, P]
     lib.oracle_quantize_pack_clip.restype = ctypes.c_int
     _lib = lib
     return lib
@@ -357,3 +369,66 @@ def kv_quantize_int4(kv: np.ndarray, group_size: int):
     q, s, _ = quantize_pack(kv.reshape(-1, d), group_size, True)
     lead = kv.shape[:-1]
     return q.reshape(*lead, d // 2), s.reshape(*lead, d // group_size)
+
+
+# ------------------------------------------------------ FP4 microscaling
+
+def e2m1_to_f32(c: int) -> float:
+    return _load().oracle_e2m1_to_f32(int(c))
+
+
+def f32_to_e2m1(v: float) -> int:
+    return _load().oracle_f32_to_e2m1(float(v))
+
+
+def e4m3_to_f32(c: int) -> float:
+    return _load().oracle_e4m3_to_f32(int(c))
+
+
+def f32_to_e4m3_sat(v: float) -> int:
+    return _load().oracle_f32_to_e4m3_sat(float(v))
+
+
+def mxfp4_quantize(W: np.ndarray):
+    """W [out, in] float32 -> (packed uint8 [out, in/2], E8M0 scale bytes [out, in/32])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    out, inn = W.shape
+    q = np.zeros((out, inn // 2), dtype=np.uint8)
+    s = np.zeros((out, inn // 32), dtype=np.uint8)
+    if _load().oracle_mxfp4_quantize(_ptr(W), out, inn, _ptr(q), _ptr(s)) != 0:
+        raise ValueError("oracle_mxfp4_quantize rejected its arguments")
+    return q, s
+
+
+def mxfp4_dequant(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    s = np.ascontiguousarray(s, dtype=np.uint8)
+    out, inn = q.shape[0], q.shape[1] * 2
+    W_hat = np.empty((out, inn), dtype=np.float32)
+    if _load().oracle_mxfp4_dequant(_ptr(q), _ptr(s), out, inn, _ptr(W_hat)) != 0:
+        raise ValueError("oracle_mxfp4_dequant rejected its arguments")
+    return W_hat
+
+
+def nvfp4_quantize(W: np.ndarray):
+    """W [out, in] float32 -> (packed uint8 [out, in/2], E4M3 scale bytes
+    [out, in/16], fp32 tensor scale)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    out, inn = W.shape
+    q = np.zeros((out, inn // 2), dtype=np.uint8)
+    s = np.zeros((out, inn // 16), dtype=np.uint8)
+    st = np.zeros(1, dtype=np.float32)
+    if _load().oracle_nvfp4_quantize(_ptr(W), out, inn, _ptr(q), _ptr(s), _ptr(st)) != 0:
+        raise ValueError("oracle_nvfp4_quantize rejected its arguments")
+    return q, s, float(st[0])
+
+
+def nvfp4_dequant(q: np.ndarray, s: np.ndarray, tensor_scale: float) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    s = np.ascontiguousarray(s, dtype=np.uint8)
+    out, inn = q.shape[0], q.shape[1] * 2
+    W_hat = np.empty((out, inn), dtype=np.float32)
+    if _load().oracle_nvfp4_dequant(_ptr(q), _ptr(s), float(tensor_scale), out, inn,
+                                    _ptr(W_hat)) != 0:
+        raise ValueError("oracle_nvfp4_dequant rejected its arguments")
+    return W_hat

@@ -543,3 +543,165 @@ ORACLE_API int oracle_kv_dequant_int8(const int8_t* codes, const uint16_t* scale
     }
     return 0;
 }
+
+/* ------------------------------------------- FP4 microscaling formats */
+
+/*
+ * E2M1 ("post-training-quantization-gptq-awq-and-rotation" (arganzheng.life)
+ * section 九.1, format table): 1 sign, 2 exponent, 1 mantissa bit; the
+ * magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6}.  A code is sign << 3 | m with
+ * magnitude index m in 0..7 in that order.
+ */
+static const float kE2M1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+ORACLE_API float oracle_e2m1_to_f32(uint8_t c) {
+    float m = kE2M1[c & 7u];
+    return (c & 8u) ? -m : m;
+}
+
+/* Nearest E2M1 value of a finite fp32 value, ties to the even magnitude
+ * index (mantissa bit 0), magnitudes above 6 saturating to 6; the sign is
+ * kept, so small negative values give -0 (code 8).  NaN gives +0. */
+ORACLE_API uint8_t oracle_f32_to_e2m1(float v) {
+    if (v != v) return 0;
+    uint8_t sign = (v < 0.0f || (v == 0.0f && signbit(v))) ? 8u : 0u;
+    double a = fabs((double)v);
+    if (a >= 6.0) return (uint8_t)(sign | 7u);
+    uint8_t best = 0;
+    for (uint8_t m = 1; m < 8; ++m) {
+        double dm = fabs(a - (double)kE2M1[m]);
+        double db = fabs(a - (double)kE2M1[best]);
+        if (dm < db || (dm == db && (m & 1u) == 0u)) best = m;
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no
+ * infinities, 0x7F / 0xFF NaN, largest finite 448, subnormals m * 2^-9). */
+ORACLE_API float oracle_e4m3_to_f32(uint8_t c) {
+    uint32_t e = (c >> 3) & 0xFu, m = c & 7u;
+    float mag;
+    if (e == 0xFu && m == 7u) mag = NAN;
+    else if (e == 0) mag = ldexpf((float)m, -9);
+    else mag = ldexpf((float)(8u | m), (int)e - 10);
+    return (c & 0x80u) ? -mag : mag;
+}
+
+/* Nearest E4M3 value of a non-negative finite fp32 value, ties to even,
+ * saturating at 448 (the block scales are never negative). */
+ORACLE_API uint8_t oracle_f32_to_e4m3_sat(float v) {
+    if (!(v > 0.0f)) return 0;
+    if (v >= 448.0f) return 0x7E;
+    uint8_t best = 0;
+    double bd = fabs((double)v);
+    for (uint32_t c = 1; c <= 0x7E; ++c) {
+        double d = fabs((double)v - (double)oracle_e4m3_to_f32((uint8_t)c));
+        if (d < bd || (d == bd && (c & 1u) == 0u)) { best = (uint8_t)c; bd = d; }
+    }
+    return best;
+}
+
+/* floor(log2(a)) of a positive finite fp32 value, exactly. */
+static int floor_log2_f32(float a) {
+    int e;
+    (void)frexpf(a, &e);          /* a = f * 2^e, f in [0.5, 1) */
+    return e - 1;
+}
+
+/*
+ * MXFP4 ("post-training-quantization-gptq-awq-and-rotation" section 九.1 and
+ * 九.2: E2M1 elements with one E8M0 power-of-two scale per 32, the OCP
+ * standard; the scale rule is the OCP one): per block of 32 consecutive
+ * elements of a row,
+ *   e = clamp(floor(log2(max |v|)) - 2, -127, 127)   (2 = E2M1's largest exponent)
+ *   X = 2^e,  scale byte = e + 127,  q = e2m1(v / X) (saturating at 6),
+ * and an all-zero block gets scale byte 0 and codes +0.  Codes packed two
+ * per byte, even element in the low nibble.
+ *   W [out, in] fp32;  packed [out, in/2];  scales [out, in/32] E8M0 bytes.
+ */
+ORACLE_API int oracle_mxfp4_quantize(const float* W, int64_t out, int64_t in, uint8_t* packed,
+                                     uint8_t* scales) {
+    if (out < 0 || in <= 0 || (in % 32) != 0) return -1;
+    uint8_t codes[32];
+    for (int64_t r = 0; r < out; ++r) {
+        for (int64_t b = 0; b < in / 32; ++b) {
+            const float* v = W + r * in + b * 32;
+            float a = 0.0f;
+            for (int k = 0; k < 32; ++k) if (fabsf(v[k]) > a) a = fabsf(v[k]);
+            int e = -127;
+            if (a > 0.0f) {
+                e = floor_log2_f32(a) - 2;
+                if (e < -127) e = -127;
+                if (e > 127) e = 127;
+            }
+            for (int k = 0; k < 32; ++k)
+                codes[k] = (a > 0.0f) ? oracle_f32_to_e2m1(ldexpf(v[k], -e)) : 0u;
+            scales[r * (in / 32) + b] = (uint8_t)(e + 127);
+            for (int k = 0; k < 32; k += 2)
+                packed[r * (in / 2) + b * 16 + k / 2] = (uint8_t)(codes[k] | (codes[k + 1] << 4));
+        }
+    }
+    return 0;
+}
+
+/* w_hat = e2m1(q) * 2^(scale - 127) in fp32 (exact). */
+ORACLE_API int oracle_mxfp4_dequant(const uint8_t* packed, const uint8_t* scales, int64_t out,
+                                    int64_t in, float* W_hat) {
+    if (out < 0 || in <= 0 || (in % 32) != 0) return -1;
+    for (int64_t r = 0; r < out; ++r)
+        for (int64_t k = 0; k < in; ++k) {
+            uint8_t byte = packed[r * (in / 2) + k / 2];
+            uint8_t c = (k & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+            int e = (int)scales[r * (in / 32) + k / 32] - 127;
+            W_hat[r * in + k] = ldexpf(oracle_e2m1_to_f32(c), e);
+        }
+    return 0;
+}
+
+/*
+ * NVFP4 (the same section: E2M1 elements, one E4M3 scale per 16 and one fp32
+ * scale per tensor).  Readings: the tensor scale maps the largest block scale
+ * amax/6 onto E4M3's largest value 448, and each block scale is amax_b / 6
+ * expressed in units of the tensor scale, all in fp32 IEEE arithmetic:
+ *   s_t = A / 2688  (A = max |W| over the tensor; 2688 = 6 * 448; s_t = 1 if A = 0)
+ *   c_b = e4m3_sat(fp32(amax_b / 6) / s_t),   S_b = fp32(e4m3(c_b) * s_t)
+ *   q = e2m1(v / S_b) (saturating at 6), codes 0 where S_b = 0,
+ * and w_hat = fp32(e2m1(q) * S_b).
+ *   packed [out, in/2];  scales [out, in/16] E4M3 bytes;  *tensor_scale fp32.
+ */
+ORACLE_API int oracle_nvfp4_quantize(const float* W, int64_t out, int64_t in, uint8_t* packed,
+                                     uint8_t* scales, float* tensor_scale) {
+    if (out < 0 || in <= 0 || (in % 16) != 0) return -1;
+    float A = 0.0f;
+    for (int64_t i = 0; i < out * in; ++i) if (fabsf(W[i]) > A) A = fabsf(W[i]);
+    const float st = (A > 0.0f) ? A / 2688.0f : 1.0f;
+    *tensor_scale = st;
+    uint8_t codes[16];
+    for (int64_t r = 0; r < out; ++r) {
+        for (int64_t b = 0; b < in / 16; ++b) {
+            const float* v = W + r * in + b * 16;
+            float a = 0.0f;
+            for (int k = 0; k < 16; ++k) if (fabsf(v[k]) > a) a = fabsf(v[k]);
+            const uint8_t cb = oracle_f32_to_e4m3_sat((a / 6.0f) / st);
+            const float S = oracle_e4m3_to_f32(cb) * st;
+            for (int k = 0; k < 16; ++k) codes[k] = (S > 0.0f) ? oracle_f32_to_e2m1(v[k] / S) : 0u;
+            scales[r * (in / 16) + b] = cb;
+            for (int k = 0; k < 16; k += 2)
+                packed[r * (in / 2) + b * 8 + k / 2] = (uint8_t)(codes[k] | (codes[k + 1] << 4));
+        }
+    }
+    return 0;
+}
+
+ORACLE_API int oracle_nvfp4_dequant(const uint8_t* packed, const uint8_t* scales,
+                                    float tensor_scale, int64_t out, int64_t in, float* W_hat) {
+    if (out < 0 || in <= 0 || (in % 16) != 0) return -1;
+    for (int64_t r = 0; r < out; ++r)
+        for (int64_t k = 0; k < in; ++k) {
+            uint8_t byte = packed[r * (in / 2) + k / 2];
+            uint8_t c = (k & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+            const float S = oracle_e4m3_to_f32(scales[r * (in / 16) + k / 16]) * tensor_scale;
+            W_hat[r * in + k] = oracle_e2m1_to_f32(c) * S;
+        }
+    return 0;
+}
