@@ -306,6 +306,60 @@ def kv_cache_cost(q4, wl, torch, device, stream, hbm_peak):
             "int8_dequant_frac": round(b_q8 / t_d8 / 1e3 / hbm_peak, 4)}
 
 
+def fp4_cost(q4, wl, torch, device, stream, hbm_peak):
+    """MXFP4 and NVFP4 quantization of the Llama-3-70B gate_proj (28672 x 8192
+    fp16, 470 MB) and their dequantization to bf16, graph-timed over two
+    rotating copies; and the weight MSE of both formats beside symmetric INT4
+    at group 32 (the same 4.5 bits per weight as NVFP4) on these N(0, 0.02^2)
+    weights.  Algorithmic bytes: fp16 in + codes + scale bytes out (dequant:
+    codes + scales in, bf16 out)."""
+    out, inn = wl.LLAMA3_70B["gate_proj"]
+    Ws = [wl.normal_weight(out, inn, 80 + i, device=device) for i in range(2)]
+    mx = [q4.mxfp4_quantize(W) for W in Ws]
+    nv = [q4.nvfp4_quantize(W) for W in Ws]
+    o16 = torch.empty(out, inn, dtype=torch.bfloat16, device=device)
+    lib = q4.load_library()
+
+    def mxq(i):
+        w = mx[i % 2]
+        lib.mxfp4_quantize(Ws[i % 2].data_ptr(), q4.Q4_F16, out, inn, w.packed.data_ptr(),
+                           w.scales.data_ptr(), torch.cuda.current_stream().cuda_stream)
+
+    def nvq(i):
+        w = nv[i % 2]
+        lib.nvfp4_quantize(Ws[i % 2].data_ptr(), q4.Q4_F16, out, inn, w.packed.data_ptr(),
+                           w.scales.data_ptr(), w.tensor_scale.data_ptr(),
+                           torch.cuda.current_stream().cuda_stream)
+
+    t_mxq = graph_time_us(torch, mxq, 8, stream)
+    t_nvq = graph_time_us(torch, nvq, 8, stream)
+    t_mxd = graph_time_us(torch, lambda i: q4.fp4_dequant(mx[i % 2], W_hat=o16), 8, stream)
+    t_nvd = graph_time_us(torch, lambda i: q4.fp4_dequant(nv[i % 2], W_hat=o16), 8, stream)
+    W = Ws[0]
+    mse = lambda What: (What.float() - W.float()).pow(2).mean().item()
+    e_mx = mse(q4.fp4_dequant(mx[0]))
+    e_nv = mse(q4.fp4_dequant(nv[0]))
+    e_i4 = mse(q4.q4_dequant(q4.q4_quantize_pack(W, 32, True)))
+    st = q4.q4_sync_status()
+    assert st == q4.Q4_OK, q4.status_string(st)
+    n = out * inn
+    b_mxq, b_nvq = 2 * n + n // 2 + n // 32, 2 * 2 * n + n // 2 + n // 16
+    b_mxd, b_nvd = n // 2 + n // 32 + 2 * n, n // 2 + n // 16 + 2 * n
+    g = lambda b, t: round(b / t / 1e3, 1)
+    del Ws, mx, nv, o16
+    return {"shape": f"{out}x{inn} fp16",
+            "mxfp4_quantize_us": round(t_mxq, 2), "mxfp4_quantize_gbs": g(b_mxq, t_mxq),
+            "nvfp4_quantize_us": round(t_nvq, 2), "nvfp4_quantize_gbs": g(b_nvq, t_nvq),
+            "nvfp4_quantize_bytes_note": "two reads of W (tensor amax, then the codes)",
+            "mxfp4_dequant_us": round(t_mxd, 2), "mxfp4_dequant_gbs": g(b_mxd, t_mxd),
+            "nvfp4_dequant_us": round(t_nvd, 2), "nvfp4_dequant_gbs": g(b_nvd, t_nvd),
+            "weight_mse": {"int4_sym_g32": e_i4, "mxfp4": e_mx, "nvfp4": e_nv},
+            "frac_of_measured_hbm": {"mxfp4_quantize": round(b_mxq / t_mxq / 1e3 / hbm_peak, 4),
+                                     "nvfp4_quantize": round(b_nvq / t_nvq / 1e3 / hbm_peak, 4),
+                                     "mxfp4_dequant": round(b_mxd / t_mxd / 1e3 / hbm_peak, 4),
+                                     "nvfp4_dequant": round(b_nvd / t_nvd / 1e3 / hbm_peak, 4)}}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -495,6 +549,7 @@ def run_ours(args):
             out["act_order"] = act_order_cost(q4, wl, torch, device, stream)
             out["w8a16"] = w8a16_cost(q4, wl, torch, device, stream, peak)
             out["kv_cache"] = kv_cache_cost(q4, wl, torch, device, stream, peak)
+            out["fp4"] = fp4_cost(q4, wl, torch, device, stream, peak)
         out["cpu_baseline"] = cpu_baseline() if (world == 1 and not args.no_cpu_baseline) else None
         print(json.dumps(out), flush=True)
     del graph

@@ -322,6 +322,51 @@ Q4_API q4_status q8_gemv(const int8_t* qweight, const float* scales, int64_t out
                          const void* x, q4_dtype x_dtype, int64_t B, void* y, q4_dtype y_dtype,
                          void* workspace, size_t workspace_bytes, q4_stream stream);
 
+/* ------------------------------------------------------ FP4 microscaling
+ *
+ * "post-training-quantization-gptq-awq-and-rotation" (arganzheng.life),
+ * sections 九.1 and 九.2: E2M1 elements {0, 0.5, 1, 1.5, 2, 3, 4, 6} x sign
+ * with a small-block scale.  Codes are packed two per byte, the even element
+ * in the low nibble; a code is sign << 3 | magnitude index; rounding is to
+ * the nearest E2M1 value with ties to the even magnitude index, saturating at
+ * 6 and keeping the sign (-0 is code 8).
+ *
+ * MXFP4 (one E8M0 power-of-two scale per 32 elements, the OCP rule):
+ *   e = clamp(floor(log2(max |v|)) - 2, -127, 127), scale byte e + 127,
+ *   q = e2m1(v * 2^-e); an all-zero block gets scale byte 0 and codes +0.
+ *   W       [out, in] fp16 or bf16, 16-byte aligned; in a multiple of 32
+ *   packed  [out, in/2] uint8, 4-byte aligned (written)
+ *   scales  [out, in/32] E8M0 bytes (written)
+ */
+Q4_API q4_status mxfp4_quantize(const void* W, q4_dtype w_dtype, int64_t out, int64_t in,
+                                uint8_t* packed, uint8_t* scales, q4_stream stream);
+
+/* w_hat = e2m1(q) * 2^(scale - 127), exact in fp32, written as out_dtype
+ * (W_hat [out, in], 16-byte aligned). */
+Q4_API q4_status mxfp4_dequant(const uint8_t* packed, const uint8_t* scales, int64_t out,
+                               int64_t in, void* W_hat, q4_dtype out_dtype, q4_stream stream);
+
+/* NVFP4 (one E4M3 scale per 16 elements and one fp32 scale per tensor):
+ *   s_t = A / 2688 (A = max |W| over the tensor; 2688 = 6 * 448; 1 if A = 0),
+ *   c_b = e4m3(fp32(amax_b / 6) / s_t) rounded to nearest even, saturating
+ *   at 448; S_b = fp32(e4m3(c_b) * s_t); q = e2m1(v / S_b) (IEEE fp32
+ *   division), codes 0 where S_b = 0.
+ *   W             [out, in] fp16 or bf16, 16-byte aligned; in a multiple of 16
+ *   packed        [out, in/2] uint8, 4-byte aligned (written)
+ *   scales        [out, in/16] E4M3 bytes (written)
+ *   tensor_scale  one fp32 in device memory, 4-byte aligned (written; used as
+ *                 scratch for the tensor maximum while the call runs)
+ */
+Q4_API q4_status nvfp4_quantize(const void* W, q4_dtype w_dtype, int64_t out, int64_t in,
+                                uint8_t* packed, uint8_t* scales, float* tensor_scale,
+                                q4_stream stream);
+
+/* w_hat = fp32(e2m1(q) * S_b) with S_b = fp32(e4m3(c_b) * s_t), written as
+ * out_dtype (W_hat [out, in], 16-byte aligned; tensor_scale a device pointer). */
+Q4_API q4_status nvfp4_dequant(const uint8_t* packed, const uint8_t* scales,
+                               const float* tensor_scale, int64_t out, int64_t in, void* W_hat,
+                               q4_dtype out_dtype, q4_stream stream);
+
 /* --------------------------------------------------------------- KV cache
  *
  * A KV cache [batch, heads, seq, head_dim] in fp16 or bf16 is passed as

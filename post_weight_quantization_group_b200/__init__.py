@@ -42,6 +42,7 @@ ABI_SYMBOLS = (
     "q4_workspace_bytes", "q4_gemv_noalloc", "q4_quantize_pack_clip", "q4_quantize_pack_perm",
     "q4_permute_activations", "q8_quantize_per_channel", "q8_dequant", "q8_workspace_bytes",
     "q8_gemv", "kv_quantize_int8", "kv_dequant_int8", "kv_quantize_int4", "kv_dequant_int4",
+    "mxfp4_quantize", "mxfp4_dequant", "nvfp4_quantize", "nvfp4_dequant",
 )
 
 
@@ -107,12 +108,17 @@ def load_library(path: str = LIB_PATH):
     lib.kv_dequant_int8.argtypes = [P, P, S, I64, I64, P, P]
     lib.kv_quantize_int4.argtypes = [P, S, I64, I64, I32, P, P, P]
     lib.kv_dequant_int4.argtypes = [P, P, I64, I64, I32, P, S, P]
+    lib.mxfp4_quantize.argtypes = [P, S, I64, I64, P, P, P]
+    lib.mxfp4_dequant.argtypes = [P, P, I64, I64, P, S, P]
+    lib.nvfp4_quantize.argtypes = [P, S, I64, I64, P, P, P, P]
+    lib.nvfp4_dequant.argtypes = [P, P, P, I64, I64, P, S, P]
     for f in ("q4_quantize_pack", "q4_quantize_pack_clip", "q4_quantize_pack_perm",
               "q4_permute_activations", "q4_dequant", "q4_gemv",
               "q4_gemm_skinny", "q4_gemv_noalloc",
               "bf16_gemv_ref_bw", "q4_sync_status", "q4_selftest_wait_timeout",
               "q8_quantize_per_channel", "q8_dequant", "q8_gemv", "kv_quantize_int8",
-              "kv_dequant_int8", "kv_quantize_int4", "kv_dequant_int4"):
+              "kv_dequant_int8", "kv_quantize_int4", "kv_dequant_int4", "mxfp4_quantize",
+              "mxfp4_dequant", "nvfp4_quantize", "nvfp4_dequant"):
         getattr(lib, f).restype = S
     lib.q4_status_string.argtypes = [S]
     lib.q4_status_string.restype = ctypes.c_char_p
@@ -507,3 +513,61 @@ def kv_dequant_int4(packed: torch.Tensor, scales: torch.Tensor, group_size: int 
                              _DT[out.dtype], _stream(stream))
     _check(st, "kv_dequant_int4")
     return out
+
+
+# ------------------------------------------------------ FP4 microscaling
+
+@dataclass
+class FP4Weight:
+    """MXFP4 (block 32, E8M0 scales) or NVFP4 (block 16, E4M3 scales and an
+    fp32 tensor scale) codes [out, in/2] uint8 with scale bytes [out, in/block]."""
+    packed: torch.Tensor
+    scales: torch.Tensor
+    out: int
+    in_features: int
+    fmt: str                                  # "mxfp4" or "nvfp4"
+    tensor_scale: torch.Tensor | None = None  # fp32 [1] on the device (NVFP4)
+
+    @property
+    def nbytes(self) -> int:
+        return self.packed.numel() + self.scales.numel() + (4 if self.tensor_scale is not None else 0)
+
+
+def mxfp4_quantize(W: torch.Tensor, stream=None) -> FP4Weight:
+    lib = load_library()
+    if W.dim() != 2 or W.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("W must be a 2-D fp16 or bf16 tensor")
+    out, inn = W.shape
+    packed = torch.empty(out, inn // 2, dtype=torch.uint8, device=W.device)
+    scales = torch.empty(out, inn // 32, dtype=torch.uint8, device=W.device)
+    _check(lib.mxfp4_quantize(_ptr(W), _DT[W.dtype], out, inn, _ptr(packed), _ptr(scales),
+                              _stream(stream)), "mxfp4_quantize")
+    return FP4Weight(packed, scales, out, inn, "mxfp4")
+
+
+def nvfp4_quantize(W: torch.Tensor, stream=None) -> FP4Weight:
+    lib = load_library()
+    if W.dim() != 2 or W.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("W must be a 2-D fp16 or bf16 tensor")
+    out, inn = W.shape
+    packed = torch.empty(out, inn // 2, dtype=torch.uint8, device=W.device)
+    scales = torch.empty(out, inn // 16, dtype=torch.uint8, device=W.device)
+    ts = torch.empty(1, dtype=torch.float32, device=W.device)
+    _check(lib.nvfp4_quantize(_ptr(W), _DT[W.dtype], out, inn, _ptr(packed), _ptr(scales),
+                              _ptr(ts), _stream(stream)), "nvfp4_quantize")
+    return FP4Weight(packed, scales, out, inn, "nvfp4", ts)
+
+
+def fp4_dequant(w: FP4Weight, out_dtype=torch.float32, W_hat: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    lib = load_library()
+    if W_hat is None:
+        W_hat = torch.empty(w.out, w.in_features, dtype=out_dtype, device=w.packed.device)
+    if w.fmt == "mxfp4":
+        st = lib.mxfp4_dequant(_ptr(w.packed), _ptr(w.scales), w.out, w.in_features, _ptr(W_hat),
+                               _DT[W_hat.dtype], _stream(stream))
+    else:
+        st = lib.nvfp4_dequant(_ptr(w.packed), _ptr(w.scales), _ptr(w.tensor_scale), w.out,
+                               w.in_features, _ptr(W_hat), _DT[W_hat.dtype], _stream(stream))
+    _check(st, f"{w.fmt}_dequant")
+    return W_hat

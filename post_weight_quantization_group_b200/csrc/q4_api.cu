@@ -1,7 +1,7 @@
 // q4_api.cu -- the C ABI of include/q4.h: argument validation, launch
 // planning, TMA descriptor encoding and kernel launches.  All kernels live in
 // this translation unit (q4_quant.cuh, q4_gemv.cuh, q4_gemv_sk.cuh,
-// q4_skinny_tc.cuh, q8_gemv.cuh, q8_quant.cuh).
+// q4_skinny_tc.cuh, q8_gemv.cuh, q8_quant.cuh, fp4_quant.cuh).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -20,6 +20,7 @@
 #include "q4_skinny_tc.cuh"
 #include "q8_gemv.cuh"
 #include "q8_quant.cuh"
+#include "fp4_quant.cuh"
 
 namespace {
 
@@ -597,6 +598,44 @@ void noalloc_mark_reclear() {
 }  // namespace
 
 // ======================================================================= ABI
+// FP4 helpers of the ABI below
+namespace {
+q4_status fp4_check_quant(const void* W, q4_dtype w_dtype, int64_t out, int64_t in, int block,
+                          const uint8_t* packed, const uint8_t* scales) {
+    if (w_dtype != Q4_F16 && w_dtype != Q4_BF16) {
+        return valid_dtype(w_dtype) ? Q4_ERR_UNSUPPORTED : Q4_ERR_INVALID_ARG;
+    }
+    if (out < 0 || in <= 0 || (in % block) != 0) return Q4_ERR_SHAPE;
+    if (out == 0) return Q4_OK;
+    if (!W || !packed || !scales) return Q4_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(packed, 4)) return Q4_ERR_ALIGNMENT;
+    return Q4_OK;
+}
+
+int fp4_blocks(int64_t nchunks, int sms) {
+    const int64_t want = (nchunks + 255) / 256;
+    return static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
+}
+
+template <bool NV>
+q4_status fp4_dequant(const uint8_t* packed, const uint8_t* scales, const float* tensor_scale,
+                      int64_t out, int64_t in, void* W_hat, q4_dtype out_dtype, cudaStream_t st) {
+    const int64_t nwords = out * in / 8;
+    const int blocks = fp4_blocks(nwords, sm_count(current_device()));
+    const uint32_t* pw = reinterpret_cast<const uint32_t*>(packed);
+    if (out_dtype == Q4_F32)
+        fp4_dequant_kernel<float, NV><<<blocks, 256, 0, st>>>(pw, scales, tensor_scale, nwords,
+                                                              reinterpret_cast<float*>(W_hat));
+    else if (out_dtype == Q4_F16)
+        fp4_dequant_kernel<__half, NV><<<blocks, 256, 0, st>>>(pw, scales, tensor_scale, nwords,
+                                                               reinterpret_cast<__half*>(W_hat));
+    else
+        fp4_dequant_kernel<__nv_bfloat16, NV><<<blocks, 256, 0, st>>>(
+            pw, scales, tensor_scale, nwords, reinterpret_cast<__nv_bfloat16*>(W_hat));
+    return launch_status(cudaSuccess);
+}
+}  // namespace
+
 extern "C" {
 
 const char* q4_version(void) { return "q4-b200 0.1 (sm_100a)"; }
@@ -1015,6 +1054,72 @@ q4_status kv_dequant_int4(const uint8_t* packed, const void* scales, int64_t row
     w.bits = 4;
     w.symmetric = 1;
     return q4_dequant(&w, out, out_dtype, stream);
+}
+
+// ------------------------------------------------------ FP4 microscaling
+
+q4_status mxfp4_quantize(const void* W, q4_dtype w_dtype, int64_t out, int64_t in,
+                         uint8_t* packed, uint8_t* scales, q4_stream stream) {
+    q4_status s = fp4_check_quant(W, w_dtype, out, in, 32, packed, scales);
+    if (s != Q4_OK || out == 0) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t nchunks = out * in / 8;
+    const int blocks = fp4_blocks(nchunks, sm_count(current_device()));
+    uint32_t* pw = reinterpret_cast<uint32_t*>(packed);
+    if (w_dtype == Q4_BF16)
+        mxfp4_quantize_kernel<true><<<blocks, 256, 0, st>>>(W, nchunks, pw, scales);
+    else
+        mxfp4_quantize_kernel<false><<<blocks, 256, 0, st>>>(W, nchunks, pw, scales);
+    return launch_status(cudaSuccess);
+}
+
+q4_status mxfp4_dequant(const uint8_t* packed, const uint8_t* scales, int64_t out, int64_t in,
+                        void* W_hat, q4_dtype out_dtype, q4_stream stream) {
+    if (!valid_dtype(out_dtype)) return Q4_ERR_INVALID_ARG;
+    if (out < 0 || in <= 0 || (in % 32) != 0) return Q4_ERR_SHAPE;
+    if (out == 0) return Q4_OK;
+    if (!packed || !scales || !W_hat) return Q4_ERR_INVALID_ARG;
+    if (!aligned(packed, 4) || !aligned(W_hat, 16)) return Q4_ERR_ALIGNMENT;
+    return fp4_dequant<false>(packed, scales, nullptr, out, in, W_hat, out_dtype,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+q4_status nvfp4_quantize(const void* W, q4_dtype w_dtype, int64_t out, int64_t in,
+                         uint8_t* packed, uint8_t* scales, float* tensor_scale,
+                         q4_stream stream) {
+    q4_status s = fp4_check_quant(W, w_dtype, out, in, 16, packed, scales);
+    if (s != Q4_OK || out == 0) return s;
+    if (!tensor_scale) return Q4_ERR_INVALID_ARG;
+    if (!aligned(tensor_scale, 4)) return Q4_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t nchunks = out * in / 8;
+    const int sms = sm_count(current_device());
+    const int blocks = fp4_blocks(nchunks, sms);
+    unsigned* amax = reinterpret_cast<unsigned*>(tensor_scale);
+    if (cudaMemsetAsync(amax, 0, sizeof(unsigned), st) != cudaSuccess) return Q4_ERR_CUDA;
+    uint32_t* pw = reinterpret_cast<uint32_t*>(packed);
+    if (w_dtype == Q4_BF16) {
+        tensor_amax_kernel<true><<<blocks, 256, 0, st>>>(W, nchunks, amax);
+        nvfp4_quantize_kernel<true><<<blocks, 256, 0, st>>>(W, nchunks, amax, pw, scales);
+    } else {
+        tensor_amax_kernel<false><<<blocks, 256, 0, st>>>(W, nchunks, amax);
+        nvfp4_quantize_kernel<false><<<blocks, 256, 0, st>>>(W, nchunks, amax, pw, scales);
+    }
+    nvfp4_finalize_kernel<<<1, 32, 0, st>>>(amax);
+    return launch_status(cudaSuccess);
+}
+
+q4_status nvfp4_dequant(const uint8_t* packed, const uint8_t* scales, const float* tensor_scale,
+                        int64_t out, int64_t in, void* W_hat, q4_dtype out_dtype,
+                        q4_stream stream) {
+    if (!valid_dtype(out_dtype)) return Q4_ERR_INVALID_ARG;
+    if (out < 0 || in <= 0 || (in % 16) != 0) return Q4_ERR_SHAPE;
+    if (out == 0) return Q4_OK;
+    if (!packed || !scales || !tensor_scale || !W_hat) return Q4_ERR_INVALID_ARG;
+    if (!aligned(packed, 4) || !aligned(W_hat, 16) || !aligned(tensor_scale, 4))
+        return Q4_ERR_ALIGNMENT;
+    return fp4_dequant<true>(packed, scales, tensor_scale, out, in, W_hat, out_dtype,
+                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 q4_status q4_selftest_wait_timeout(int64_t limit_ns, q4_stream stream) {

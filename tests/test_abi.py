@@ -271,3 +271,24 @@ def test_kv_cache_validation(lib):
     assert d4(A16, A16, 4, 128, 128, None, q4.Q4_F16, None) == q4.Q4_ERR_INVALID_ARG
     assert d4(A16, A16, 4, 128, 96, A16, q4.Q4_F16, None) == q4.Q4_ERR_SHAPE
     assert d4(A16, A16, 0, 128, 128, A16, q4.Q4_F16, None) == q4.Q4_OK
+
+
+def test_fp4_validation(lib):
+    mq = lib.mxfp4_quantize
+    assert mq(A16, q4.Q4_F32, 4, 64, A16, A16, None) == q4.Q4_ERR_UNSUPPORTED
+    assert mq(A16, q4.Q4_BF16, 4, 48, A16, A16, None) == q4.Q4_ERR_SHAPE      # in % 32
+    assert mq(A16, q4.Q4_BF16, 0, 64, A16, A16, None) == q4.Q4_OK
+    assert mq(A2, q4.Q4_BF16, 4, 64, A16, A16, None) == q4.Q4_ERR_ALIGNMENT
+    assert mq(A16, q4.Q4_BF16, 4, 64, None, A16, None) == q4.Q4_ERR_INVALID_ARG
+    nq = lib.nvfp4_quantize
+    assert nq(A16, q4.Q4_BF16, 4, 40, A16, A16, A16, None) == q4.Q4_ERR_SHAPE  # in % 16
+    assert nq(A16, q4.Q4_BF16, 4, 64, A16, A16, None, None) == q4.Q4_ERR_INVALID_ARG
+    assert nq(A16, q4.Q4_BF16, 4, 64, A16, A16, A2, None) == q4.Q4_ERR_ALIGNMENT
+    assert nq(A16, q4.Q4_BF16, 0, 64, A16, A16, A16, None) == q4.Q4_OK
+    md = lib.mxfp4_dequant
+    assert md(A16, A16, 4, 64, A16, 9, None) == q4.Q4_ERR_INVALID_ARG
+    assert md(A16, A16, 4, 48, A16, q4.Q4_F32, None) == q4.Q4_ERR_SHAPE
+    assert md(A16, A16, 4, 64, A2, q4.Q4_F32, None) == q4.Q4_ERR_ALIGNMENT
+    nd = lib.nvfp4_dequant
+    assert nd(A16, A16, None, 4, 64, A16, q4.Q4_F32, None) == q4.Q4_ERR_INVALID_ARG
+    assert nd(A16, A16, A16, 0, 64, A16, q4.Q4_F32, None) == q4.Q4_OK
