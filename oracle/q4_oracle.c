@@ -35,6 +35,10 @@
  *    [-127, 127]: charles2530.github.io, section 13 (快速代码示例).
  *  - INT8 KV cache, one scale per token row of head_dim values, codes in
  *    [-128, 127], and its dequantization: "压缩算法" section 7.4.1.1.
+ *  - E2M1, E4M3, MXFP4 (E8M0 scale per 32, the OCP rule) and NVFP4 (E4M3
+ *    scale per 16 and an fp32 tensor scale): arganzheng.life sections 九.1
+ *    and 九.2 (the scale choices and E2M1 rounding are readings, stated with
+ *    the functions below).
  *
  * Readings taken where the pages leave a step open:
  *  - the scale is computed in fp32 (IEEE division), stored as fp16, and the
