@@ -244,6 +244,49 @@ def act_order_cost(q4, wl, torch, device, stream):
             "overhead": round(t_both / t_prod - 1.0, 4)}
 
 
+def fused_layer_cost(q4, wl, torch, device, stream, layers, steps, hbm_peak):
+    """The same Llama-3-8B step with q/k/v and gate/up stored as one matrix
+    each ([6144, 4096] and [28672, 4096], rows concatenated before
+    quantization, as serving engines lay them out): 4 products per layer
+    instead of 7, the same weights, codes and bytes (row-wise quantization
+    gives the same codes).  Graph-timed like the headline step."""
+    mats = []
+    for layer in range(layers):
+        seeds = wl.llama3_8b_layer_seeds(layer)
+        W = {name: wl.normal_weight(out, inn, seeds[name], device=device)
+             for name, (out, inn) in wl.LLAMA3_8B.items()}
+        for name, parts in (("qkv", ("q_proj", "k_proj", "v_proj")), ("o", ("o_proj",)),
+                            ("gate_up", ("gate_proj", "up_proj")), ("down", ("down_proj",))):
+            Wc = torch.cat([W[p] for p in parts], dim=0)
+            mats.append((name, q4.q4_quantize_pack(Wc, 128, True)))
+            del Wc
+        del W
+    xs = {4096: wl.activations(1, 4096, 17 + 4096, device=device),
+          14336: wl.activations(1, 14336, 17 + 14336, device=device)}
+    ys = {name: torch.empty(1, w.out, dtype=torch.bfloat16, device=device) for name, w in mats[:4]}
+    step_bytes = sum(algo_bytes(w.out, w.in_features, 128, 1) for _, w in mats)
+
+    def step():
+        for name, w in mats:
+            q4.q4_gemv(w, xs[w.in_features], y=ys[name])
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+        step()
+    n = max(20, steps // 4)
+    ms = time_region(torch, graph.replay, n, 3, stream) / n
+    st = q4.q4_sync_status()
+    assert st == q4.Q4_OK, q4.status_string(st)
+    del graph, mats
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    return {"layout": "q/k/v and gate/up fused row-wise, 4 products per layer",
+            "us_per_layer": round(ms * 1e3 / layers, 3), "gbs": round(gbs, 1),
+            "frac_of_measured_hbm": round(gbs / hbm_peak, 4), "bytes_per_step": step_bytes}
+
+
 def w8a16_cost(q4, wl, torch, device, stream, hbm_peak):
     """Per-channel INT8 W8A16 product (q8_gemv) on the Llama-3-70B down_proj
     and gate_proj shapes at B = 1 and 8, beside the INT4 product (sym g128)
@@ -547,6 +590,8 @@ def run_ours(args):
         if world == 1 and not args.no_sweep:
             out["int4_vs_bf16_by_B"] = b_sweep(q4, wl, torch, device, stream)
             out["act_order"] = act_order_cost(q4, wl, torch, device, stream)
+            out["fused_qkv_gate_up"] = fused_layer_cost(q4, wl, torch, device, stream, layers,
+                                                         args.steps, peak)
             out["w8a16"] = w8a16_cost(q4, wl, torch, device, stream, peak)
             out["kv_cache"] = kv_cache_cost(q4, wl, torch, device, stream, peak)
             out["fp4"] = fp4_cost(q4, wl, torch, device, stream, peak)

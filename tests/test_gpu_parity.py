@@ -538,3 +538,9 @@ def test_act_order_bad_index_is_reported():
     assert q4.q4_sync_status() == q4.Q4_ERR_INVALID_ARG
     assert q4.q4_sync_status() == q4.Q4_OK
     _gemv_case(256, 1024, 128, True, 2, torch.bfloat16)  # still usable
+
+
+@pytest.mark.parametrize("shape", [(6144, 4096), (28672, 4096)])
+def test_gemv_fused_qkv_and_gate_up_shapes(shape):
+    """The Llama-3-8B q/k/v and gate/up matrices stored row-concatenated."""
+    _gemv_case(*shape, 128, True, 1, torch.bfloat16, seed=40, rows=_sample_rows(shape[0], 160))
