@@ -779,7 +779,9 @@ def run_reference(args):
 def run_op(args):
     """One operation of the path alone, for profiling and spot timing:
     ``w8a16-70b`` = q8_gemv on the Llama-3-70B down_proj (8192 x 28672, batch
-    --batch, two weight copies rotating); ``kv8-70b-32k`` = kv_quantize_int8
+    --batch, two weight copies rotating); ``q4-70b-down`` = q4_gemm_skinny
+    (sym g128) on the same shape and batch (the B <= 8 kernel or, above, the
+    tcgen05 kernel); ``kv8-70b-32k`` = kv_quantize_int8
     of one layer's K cache at 32768 tokens ([1, 8, 32768, 128] bf16, four
     caches rotating).  Prints one JSON line (CUDA-event time per call)."""
     import torch
@@ -805,6 +807,19 @@ def run_op(args):
         fn = lambda: q4.q8_gemv(ws[next(it) % 2], x, y=y, workspace=wsp)
         nbytes = out * inn + out * 4 + B * inn * 2 + B * out * 2
         name, cfg = "W8A16 per-channel INT8 GEMV", {"workload": f"Llama-3-70B down_proj {out}x{inn}", "batch": B}
+    elif args.workload == "q4-70b-down":
+        out, inn = wl.LLAMA3_70B["down_proj"]
+        B = args.batch
+        ws = [q4.q4_quantize_pack(wl.normal_weight(out, inn, 30 + i, device=device), 128, True)
+              for i in range(2)]
+        torch.cuda.empty_cache()
+        x = wl.activations(B, inn, 31, device=device)
+        y = torch.empty(B, out, dtype=torch.bfloat16, device=device)
+        wsp = q4.workspace_for(ws[0], B, device)
+        it = iter(range(1 << 30))
+        fn = lambda: q4.q4_gemm_skinny(ws[next(it) % 2], x, y=y, workspace=wsp)
+        nbytes = algo_bytes(out, inn, 128, B)
+        name, cfg = "W4A16 INT4 product (sym g128)", {"workload": f"Llama-3-70B down_proj {out}x{inn}", "batch": B}
     else:
         shape = (1, wl.LLAMA3_70B_KV_HEADS, 32768, wl.LLAMA3_70B_HEAD_DIM)
         caches = [wl.kv_cache(*shape, seed=70 + i, dtype=torch.bfloat16, device=device) for i in range(4)]
@@ -834,7 +849,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama3-8b",
-                    choices=["llama3-8b", "llama3-70b-stack", "w8a16-70b", "kv8-70b-32k"])
+                    choices=["llama3-8b", "llama3-70b-stack", "w8a16-70b", "q4-70b-down",
+                             "kv8-70b-32k"])
     ap.add_argument("--batch", type=int, default=1, help="batch of the llama3-70b-stack workload")
     ap.add_argument("--layers", type=int, default=32,
                     help="distinct decoder layers per step (32 = the Llama-3-8B depth)")
@@ -849,7 +865,7 @@ def main():
         run_reference(args)
     elif args.workload == "llama3-70b-stack":
         run_stack(args)
-    elif args.workload in ("w8a16-70b", "kv8-70b-32k"):
+    elif args.workload in ("w8a16-70b", "q4-70b-down", "kv8-70b-32k"):
         run_op(args)
     else:
         run_ours(args)
