@@ -252,22 +252,21 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 // input but without the division in almost every case.  With r = 1/s
 // correctly rounded (quot_recip) and t = w * r rounded to nearest, the
 // relative errors give |t - w/s| <= |w/s| (2u + u^2) and
-// |fl(w/s) - w/s| <= |w/s| u (u = 2^-24), so t and the IEEE quotient differ
-// by less than |t| 2^-22.  The distance d from t to the nearest half-integer
-// is computed with an absolute error below 2^-24.  When d exceeds
-// |t| 2^-22 + 2^-23, t and the IEEE quotient lie strictly on the same side of
-// every half-integer and round to the same integer; otherwise (a near tie,
-// |t| >= 2^22, or a non-finite t) the exact quotient is rounded instead.
+// |fl(w/s) - w/s| <= |w/s| u (u = 2^-24), so |t - fl(w/s)| <= |t| (3u + u^2),
+// below 3.2e-5 while |t| < 178.  t - rint(t) is exact.  So when |t| < 178 and
+// |t - rint(t)| < 0.5 - 3.2e-5, t and the IEEE quotient lie strictly on the
+// same side of every half-integer and round to the same integer; otherwise
+// (a near tie, a large or non-finite t) the exact quotient is rounded.
 __device__ __forceinline__ float quot_recip(float s) {
     const float r = __frcp_rn(s);
     // a subnormal reciprocal has no 2^-24 relative error bound: take the
-    // exact path for every element (NaN t fails the distance test)
+    // exact path for every element (a NaN t fails the test below)
     return fabsf(r) >= 1.17549435e-38f ? r : __int_as_float(0x7FC00000);
 }
 __device__ __forceinline__ float rne_quot(float w, float s, float r) {
     const float t = __fmul_rn(w, r);
-    const float d = fabsf(__fsub_rn(__fsub_rn(t, floorf(t)), 0.5f));
-    if (d > __fmaf_rn(fabsf(t), 2.384185791015625e-7f, 1.1920928955078125e-7f)) return rintf(t);
+    const float q = rintf(t);
+    if (fabsf(__fsub_rn(t, q)) < 0.4999679f && fabsf(t) < 178.0f) return q;
     return rintf(__fdiv_rn(w, s));
 }
 

@@ -4,7 +4,7 @@
 // Weights ("量化：PTQ、GPTQ、AWQ 与 SmoothQuant" (charles2530.github.io)
 // section 13, per_channel_int8_quant), one scale per row of W [out, in]:
 //   s = max(max_k |w|, 1e-6) / 127,   q = clamp(rne(w / s), -127, 127)
-// in fp32 with the results of IEEE divisions (rne_quot); s is stored as fp32
+// in fp32 with the results of IEEE divisions (int8_code); s is stored as fp32
 // and w_hat = q * s.
 //
 // KV cache ("压缩算法" (cs-knowledge-wiki) section 7.4.1.1,
@@ -22,6 +22,33 @@
 namespace q4dev {
 
 // ---------------------------------------------------------- INT8 weights
+
+// INT8 code of one value, clamp(rne(fl(v / s)), qmin, 127), through t = v * r
+// (r = 1/s correctly rounded, from quot_recip): |t - fl(v/s)| <= |t| (3u + u^2)
+// (u = 2^-24), below 3.2e-5 while |t| < 178, and t - rint(t) is exact; so when
+// |t - rint(t)| < 0.5 - 3.2e-5 both round to the same integer, and from
+// |t| >= 178 on both clamp alike.  Otherwise (near a tie, or a NaN) the exact
+// quotient is rounded as the definition states (NaN -> qmin).
+__device__ __forceinline__ int int8_code(float v, float s, float r, int qmin) {
+    const float t = __fmul_rn(v, r);
+    const int q = __float2int_rn(t);
+    if (fabsf(__fsub_rn(t, __int2float_rn(q))) < 0.4999679f) return min(max(q, qmin), 127);
+    float u = rintf(__fdiv_rn(v, s));
+    u = fminf(fmaxf(u, static_cast<float>(qmin)), 127.f);
+    return static_cast<int>(u);
+}
+
+// Eight codes as two little-endian words (element 0 in byte 0).
+__device__ __forceinline__ uint2 pack8_bytes(const int (&q)[8]) {
+    uint32_t w[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t lo = __byte_perm(q[4 * h], q[4 * h + 1], 0x0040);
+        const uint32_t hi = __byte_perm(q[4 * h + 2], q[4 * h + 3], 0x0040);
+        w[h] = __byte_perm(lo, hi, 0x5410);
+    }
+    return make_uint2(w[0], w[1]);
+}
 
 // One CTA per row (grid-stride over rows): the row's amax by a block
 // reduction, then the codes; the second read of the row comes from L2.
@@ -58,15 +85,10 @@ __global__ void __launch_bounds__(256)
         for (int64_t k = static_cast<int64_t>(threadIdx.x) * 8; k < in; k += 256 * 8) {
             float v[8];
             load8_f32<BF16IN>(W, r * in + k, v);
-            uint32_t packed[2] = {0u, 0u};
+            int c[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float t = rne_quot(v[i], s, rs);
-                t = fminf(fmaxf(t, -127.f), 127.f);  // a NaN quotient becomes -127
-                const uint32_t b = static_cast<uint32_t>(static_cast<int>(t)) & 0xFFu;
-                packed[i >> 2] |= b << (8 * (i & 3));
-            }
-            *reinterpret_cast<uint2*>(q + r * in + k) = make_uint2(packed[0], packed[1]);
+            for (int i = 0; i < 8; ++i) c[i] = int8_code(v[i], s, rs, -127);
+            *reinterpret_cast<uint2*>(q + r * in + k) = pack8_bytes(c);
         }
         __syncthreads();  // red / s_row are reused by the next row
     }
@@ -131,6 +153,7 @@ __device__ __forceinline__ float cache_value(uint16_t b) {
     }
 }
 
+
 // A team of TS lanes (a power of two dividing 32) per row of d values; a lane
 // holds the 8-value vectors sub and sub + TS of the row (d <= 16 * TS).  The
 // warp's loop bound is uniform so that every lane takes part in the
@@ -169,18 +192,14 @@ __global__ void __launch_bounds__(256)
         for (int h = 0; h < 2; ++h) {
             const int vec = sub + h * TS;
             if (!(live && vec < V)) continue;
-            uint32_t packed[2] = {0u, 0u};
+            uint2 packed = make_uint2(0u, 0u);
+            if (s != 0.f) {
+                int q[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float t = 0.f;
-                if (s != 0.f) {
-                    t = rne_quot(v[h][i], s, rs);
-                    t = fminf(fmaxf(t, -128.f), 127.f);
-                }
-                const uint32_t b = static_cast<uint32_t>(static_cast<int>(t)) & 0xFFu;
-                packed[i >> 2] |= b << (8 * (i & 3));
+                for (int i = 0; i < 8; ++i) q[i] = int8_code(v[h][i], s, rs, -128);
+                packed = pack8_bytes(q);
             }
-            *reinterpret_cast<uint2*>(codes + r * d + vec * 8) = make_uint2(packed[0], packed[1]);
+            *reinterpret_cast<uint2*>(codes + r * d + vec * 8) = packed;
         }
     }
 }
