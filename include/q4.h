@@ -19,21 +19,33 @@
  *     -- arganzheng.life section 二.1 (decode GEMM [B, k] x [k, n]) and
  *        section 二.3 (W4A16 dataflow: shift, mask, x s, + z on chip).
  *
+ * Beside the INT4 path: the per-group range (clipping) search and act order
+ * of the INT4 quantizer (arganzheng.life sections 三.2, 五.3, 九.2);
+ * per-output-channel INT8 weights and their W8A16 product
+ * ("量化：PTQ、GPTQ、AWQ 与 SmoothQuant" (charles2530.github.io) section 13);
+ * INT8 and INT4 KV-cache quantization ("压缩算法" (cs-knowledge-wiki)
+ * sections 7.4.1.1-7.4.1.2); and the FP4 microscaling formats MXFP4 and
+ * NVFP4 (arganzheng.life sections 九.1-九.2).  Each is documented at its
+ * declaration below.
+ *
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - Every pointer argument is a DEVICE pointer (except `w`, the q4_weight
  *    descriptor, which is a host struct passed by pointer and read during the
  *    call only).  The caller owns all memory.  The library never allocates,
- *    frees or synchronizes (except q4_sync_status) and enqueues all of its
- *    work on `stream` (a cudaStream_t; NULL = the legacy default stream).
+ *    frees or synchronizes (except q4_sync_status and the first
+ *    q4_gemv_noalloc call per device) and enqueues all of its work on
+ *    `stream` (a cudaStream_t; NULL = the legacy default stream).
  *  - Tensors are dense and row-major.  W and W_hat are [out, in]; x is
  *    [B, in]; y is [B, out]; scales and zeros are [out, in / group_size].
  *  - Packed codes: qweight is [out, in / 2] bytes; byte j of a row holds
  *    element 2j in its low nibble and element 2j+1 in its high nibble.
  *    Symmetric codes are stored as 4-bit two's complement (q & 0xF);
  *    asymmetric codes as unsigned 4-bit integers.
- *  - Scales are fp16.  Zero points are fp16 holding integers in [0, 15];
- *    zeros == NULL if and only if symmetric.
+ *  - INT4 scales are fp16.  Zero points are fp16 holding integers in
+ *    [0, 15]; zeros == NULL if and only if symmetric.  (INT8 weights carry
+ *    fp32 row scales, KV caches scales in their own 16-bit type, FP4 formats
+ *    E8M0 / E4M3 scale bytes: see their declarations.)
  *  - Argument errors are returned synchronously and nothing is launched.
  *    Errors that happen on the device after a successful return (a bounded
  *    wait that ran out) are reported by q4_sync_status.  A CUDA launch error
