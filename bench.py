@@ -302,7 +302,7 @@ def w8a16_cost(q4, wl, torch, device, stream, hbm_peak):
         for B in (1, 8):
             x = wl.activations(B, inn, 61, device=device)
             y = torch.empty(B, out, dtype=torch.bfloat16, device=device)
-            wsp = q4._shared_workspace(int(q4.load_library().q8_workspace_bytes(out, inn, B)), device)
+            wsp = q4.q8_workspace_for(w8[0], B, device)
             t8 = graph_time_us(torch, lambda i: q4.q8_gemv(w8[i % 2], x, y=y, workspace=wsp), 16, stream)
             wsp4 = q4.workspace_for(w4[0], B, device)
             t4 = graph_time_us(torch, lambda i: q4.q4_gemv(w4[i % 2], x, y=y, workspace=wsp4), 16, stream)
@@ -802,7 +802,7 @@ def run_op(args):
         torch.cuda.empty_cache()
         x = wl.activations(B, inn, 61, device=device)
         y = torch.empty(B, out, dtype=torch.bfloat16, device=device)
-        wsp = q4._shared_workspace(int(q4.load_library().q8_workspace_bytes(out, inn, B)), device)
+        wsp = q4.q8_workspace_for(ws[0], B, device)
         it = iter(range(1 << 30))
         fn = lambda: q4.q8_gemv(ws[next(it) % 2], x, y=y, workspace=wsp)
         nbytes = out * inn + out * 4 + B * inn * 2 + B * out * 2

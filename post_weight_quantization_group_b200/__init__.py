@@ -424,6 +424,12 @@ def q8_dequant(w: Q8Weight, out_dtype=torch.float32, W_hat: torch.Tensor | None 
     return W_hat
 
 
+def q8_workspace_for(w: Q8Weight, B: int, device) -> torch.Tensor:
+    """The per-device zero-filled workspace (shared with q4_gemv) grown for
+    q8_gemv on ``w`` with batch ``B``."""
+    return _shared_workspace(int(load_library().q8_workspace_bytes(w.out, w.in_features, B)), device)
+
+
 def q8_gemv(w: Q8Weight, x: torch.Tensor, y: torch.Tensor | None = None, y_dtype=None,
             workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """y = x (q * s)^T for B <= 8 (x [B, in] bf16/fp16; y [B, out] x.dtype or fp32)."""
@@ -434,8 +440,7 @@ def q8_gemv(w: Q8Weight, x: torch.Tensor, y: torch.Tensor | None = None, y_dtype
     if y is None:
         y = torch.empty(B, w.out, dtype=y_dtype or x.dtype, device=x.device)
     if workspace is None:
-        workspace = _shared_workspace(int(lib.q8_workspace_bytes(w.out, w.in_features, B)),
-                                      x.device)
+        workspace = q8_workspace_for(w, B, x.device)
     st = lib.q8_gemv(_ptr(w.qweight), _ptr(w.scales), w.out, w.in_features, _ptr(x), _DT[x.dtype],
                      B, _ptr(y), _DT[y.dtype], _ptr(workspace),
                      workspace.numel() * workspace.element_size(), _stream(stream))
