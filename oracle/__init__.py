@@ -100,6 +100,8 @@ def _load():
     lib.oracle_mxfp4_dequant.argtypes = [P, P, I64, I64, P]
     lib.oracle_nvfp4_quantize.argtypes = [P, I64, I64, P, P, P]
     lib.oracle_nvfp4_dequant.argtypes = [P, P, ctypes.c_float, I64, I64, P]
+    lib.oracle_fp4_gemm_f64.argtypes = [P, P, ctypes.c_float, P, P, ctypes.c_float, I32, I64, I64,
+                                        I64, P]
     lib.oracle_quantize_pack_clip.restype = ctypes.c_int
     _lib = lib
     return lib
@@ -432,3 +434,20 @@ def nvfp4_dequant(q: np.ndarray, s: np.ndarray, tensor_scale: float) -> np.ndarr
                                     _ptr(W_hat)) != 0:
         raise ValueError("oracle_nvfp4_dequant rejected its arguments")
     return W_hat
+
+
+def fp4_gemm(fmt: str, wq, ws, w_st, xq, xs, x_st) -> np.ndarray:
+    """W4A4 product y [B, out] fp64 of two FP4 operands of the same format
+    (packed codes and scale bytes as mxfp4_quantize / nvfp4_quantize return
+    them; w_st, x_st the NVFP4 tensor scales, ignored for MXFP4)."""
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    ws = np.ascontiguousarray(ws, dtype=np.uint8)
+    xq = np.ascontiguousarray(np.atleast_2d(xq), dtype=np.uint8)
+    xs = np.ascontiguousarray(np.atleast_2d(xs), dtype=np.uint8)
+    out, inn, B = wq.shape[0], wq.shape[1] * 2, xq.shape[0]
+    y = np.empty((B, out), dtype=np.float64)
+    f = 0 if fmt == "mxfp4" else 1
+    if _load().oracle_fp4_gemm_f64(_ptr(wq), _ptr(ws), float(w_st or 1.0), _ptr(xq), _ptr(xs),
+                                   float(x_st or 1.0), f, out, inn, B, _ptr(y)) != 0:
+        raise ValueError("oracle_fp4_gemm_f64 rejected its arguments")
+    return y

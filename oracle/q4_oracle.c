@@ -709,3 +709,40 @@ ORACLE_API int oracle_nvfp4_dequant(const uint8_t* packed, const uint8_t* scales
         }
     return 0;
 }
+
+/*
+ * The W4A4 product of two FP4 operands (the use of the microscaling formats
+ * on Blackwell's block-scaled tensor cores, arganzheng.life sections 九.1,
+ * 九.2: FP4 puts the non-uniform grid into activation quantization too):
+ *   y[b, r] = sum_k w_hat[r, k] * x_hat[b, k]   in fp64,
+ * with w_hat, x_hat the values of the packed codes and block scales taken
+ * exactly in fp64 (e2m1 * 2^e for MXFP4; e2m1 * e4m3 * s_t for NVFP4, the
+ * product of three short significands, exact), i.e. the product a
+ * block-scaled MMA computes before its fp32 rounding.
+ *   fmt 0 = MXFP4 (scales [rows, in/32] E8M0), 1 = NVFP4 (scales [rows, in/16]
+ *   E4M3, tensor scales w_st, x_st); packed [rows, in/2].
+ */
+static double fp4_value_f64(const uint8_t* packed, const uint8_t* scales, double st, int fmt,
+                            int64_t in, int64_t r, int64_t k) {
+    uint8_t byte = packed[r * (in / 2) + k / 2];
+    uint8_t c = (k & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+    double e = (double)oracle_e2m1_to_f32(c);
+    if (fmt == 0) return ldexp(e, (int)scales[r * (in / 32) + k / 32] - 127);
+    return e * (double)oracle_e4m3_to_f32(scales[r * (in / 16) + k / 16]) * st;
+}
+
+ORACLE_API int oracle_fp4_gemm_f64(const uint8_t* wq, const uint8_t* ws, float w_st,
+                                   const uint8_t* xq, const uint8_t* xs, float x_st, int32_t fmt,
+                                   int64_t out, int64_t in, int64_t B, double* y) {
+    const int64_t blk = fmt == 0 ? 32 : 16;
+    if (out < 0 || B < 0 || in <= 0 || (in % blk) != 0 || (fmt != 0 && fmt != 1)) return -1;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t r = 0; r < out; ++r) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < in; ++k)
+                acc += fp4_value_f64(wq, ws, (double)w_st, fmt, in, r, k) *
+                       fp4_value_f64(xq, xs, (double)x_st, fmt, in, b, k);
+            y[b * out + r] = acc;
+        }
+    return 0;
+}

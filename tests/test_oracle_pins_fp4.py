@@ -154,3 +154,53 @@ def test_fp4_error_ordering_on_gaussian_weights():
     q, s, st = oracle.nvfp4_quantize(W)
     e_nv = np.mean((oracle.nvfp4_dequant(q, s, st) - W) ** 2)
     assert e_nv < e_mx
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_fp4_gemm_equals_matmul_of_dequantised(fmt):
+    """The W4A4 product equals numpy's matmul of the two dequantised
+    operands (fp32 dequantizations, exact here) and, on a weight and an
+    activation that are already FP4 grid values, the unquantised product."""
+    rng = np.random.default_rng(4)
+    W = (rng.standard_normal((24, 96)) * 0.02).astype(np.float32)
+    X = rng.standard_normal((3, 96)).astype(np.float32)
+    if fmt == "mxfp4":
+        wq, ws = oracle.mxfp4_quantize(W)
+        xq, xs = oracle.mxfp4_quantize(X)
+        wst = xst = None
+        Wd, Xd = oracle.mxfp4_dequant(wq, ws), oracle.mxfp4_dequant(xq, xs)
+    else:
+        wq, ws, wst = oracle.nvfp4_quantize(W)
+        xq, xs, xst = oracle.nvfp4_quantize(X)
+        Wd, Xd = oracle.nvfp4_dequant(wq, ws, wst), oracle.nvfp4_dequant(xq, xs, xst)
+    y = oracle.fp4_gemm(fmt, wq, ws, wst, xq, xs, xst)
+    ref = Xd.astype(np.float64) @ Wd.astype(np.float64).T
+    # NVFP4's dequantization rounds S_b = e4m3 * s_t to fp32 (relative 2^-24 per
+    # term); the product takes the scales exactly
+    assert np.allclose(y, ref, rtol=1e-6, atol=1e-6 * np.sqrt(np.mean(ref ** 2)))
+    # grid values survive quantization: the product is then the plain one
+    G = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6, -6, -4, -3, -2, -1.5, -1, -0.5, -0.0] * 2,
+                 dtype=np.float32)[None, :].repeat(2, 0)
+    H = np.roll(G, 5, axis=1)
+    if fmt == "mxfp4":
+        gq, gs = oracle.mxfp4_quantize(G)
+        hq, hs = oracle.mxfp4_quantize(H)
+        yg = oracle.fp4_gemm(fmt, gq, gs, None, hq, hs, None)
+    else:
+        gq, gs, gst = oracle.nvfp4_quantize(G)
+        hq, hs, hst = oracle.nvfp4_quantize(H)
+        yg = oracle.fp4_gemm(fmt, gq, gs, gst, hq, hs, hst)
+    assert np.allclose(yg, H.astype(np.float64) @ G.astype(np.float64).T, rtol=1e-6)
+
+
+def test_fp4_gemm_hand_block():
+    """One MXFP4 block each: w = [6, 1, 0.5, ...0] at scale 2^0, x = [1, -2, 4,
+    ...0] at scale 2^-1 -> y = 6*0.5 + 1*(-1) + 0.5*2 = 3."""
+    W = np.zeros((1, 32), dtype=np.float32)
+    W[0, :3] = [6.0, 1.0, 0.5]
+    X = np.zeros((1, 32), dtype=np.float32)
+    X[0, :3] = [0.5, -1.0, 2.0]                    # amax 2 -> e = -1, codes 1, -2, 4
+    wq, ws = oracle.mxfp4_quantize(W)
+    xq, xs = oracle.mxfp4_quantize(X)
+    assert ws[0, 0] == 127 and xs[0, 0] == 126
+    assert oracle.fp4_gemm("mxfp4", wq, ws, None, xq, xs, None)[0, 0] == 3.0
