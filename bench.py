@@ -37,11 +37,12 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# DRAM traffic of q4_gemv_sk_kernel per algorithmic byte, from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum = 30.33 MB on a 14336 x 4096
-# gate_proj launch whose algorithmic bytes are 30.28 MB; same ratio in every
-# capture of this kernel so far).  Scaled to the
-# bench's average launch; it must be re-taken whenever the kernel changes.
+# DRAM traffic of q4_gemv_sk_kernel per algorithmic byte, from the ncu capture
+# of a launch of this workload (dram__bytes_read.sum + dram__bytes_write.sum =
+# 30.33 MB on a 14336 x 4096 gate_proj launch whose algorithmic bytes are
+# 30.28 MB).  Shapes with few row tiles write stream-K partials too (the
+# 70B down_proj capture: reads 1.018x, plus 3.8 MB of partials).  Scaled to
+# the bench's average launch; it must be re-taken whenever the kernel changes.
 GEMV_TRAFFIC_RATIO = 30.33 / 30.28
 GEMV_TRAFFIC_SOURCE = ("ncu --set full on one 14336x4096 B=1 launch of the current kernel "
                        "(profiles/q4_gemv_sk_llama3_8b_gate_full.txt), scaled by algorithmic bytes")
