@@ -292,3 +292,17 @@ def test_fp4_validation(lib):
     nd = lib.nvfp4_dequant
     assert nd(A16, A16, None, 4, 64, A16, q4.Q4_F32, None) == q4.Q4_ERR_INVALID_ARG
     assert nd(A16, A16, A16, 0, 64, A16, q4.Q4_F32, None) == q4.Q4_OK
+
+
+def test_c_consumer_compiles_links_and_runs(lib, tmp_path):
+    """A plain C99 program built against include/q4.h and linked with
+    libq4.so runs its host-side checks (no GPU needed)."""
+    import subprocess
+    exe = tmp_path / "abi_from_c"
+    libdir = os.path.dirname(q4.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c", "abi_from_c.c"), "-L", libdir, "-l:libq4.so",
+                    f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stderr
+    assert "c abi ok" in out.stdout
