@@ -400,12 +400,12 @@ __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
                     const uint32_t a = w0[i], b = w1[i];
                     const uint32_t A0[4] = {lop3_and_xor(a, 0x000F000Fu, kMagic),
                                             lop3_and_xor(b, 0x000F000Fu, kMagic),
-                                            lop3_and_xor(shr_fma<4>(a), 0x000F000Fu, kMagic),
-                                            lop3_and_xor(shr_fma<4>(b), 0x000F000Fu, kMagic)};
-                    const uint32_t A1[4] = {lop3_and_xor(shr_fma<8>(a), 0x000F000Fu, kMagic),
-                                            lop3_and_xor(shr_fma<8>(b), 0x000F000Fu, kMagic),
-                                            lop3_and_xor(shr_fma<12>(a), 0x000F000Fu, kMagic),
-                                            lop3_and_xor(shr_fma<12>(b), 0x000F000Fu, kMagic)};
+                                            lop3_and_xor((a >> 4), 0x000F000Fu, kMagic),
+                                            lop3_and_xor((b >> 4), 0x000F000Fu, kMagic)};
+                    const uint32_t A1[4] = {lop3_and_xor((a >> 8), 0x000F000Fu, kMagic),
+                                            lop3_and_xor((b >> 8), 0x000F000Fu, kMagic),
+                                            lop3_and_xor((a >> 12), 0x000F000Fu, kMagic),
+                                            lop3_and_xor((b >> 12), 0x000F000Fu, kMagic)};
                     mma_16816<BF16>(pa, A0, xf[i][0], xf[i][1]);
                     mma_16816<BF16>(pb, A1, xf[i][2], xf[i][3]);
                 }
