@@ -262,10 +262,12 @@ Q4_API q4_status q4_gemm_skinny(const q4_weight* w, const void* x, q4_dtype x_dt
  * Q4_ERR_WORKSPACE before anything is launched.  No device memory is
  * allocated or freed, by the library or by anything it calls.
  *
- * The first call on each device does setup: with that device current it
- * looks up the scratch address (a failure returns Q4_ERR_CUDA), zero-fills
- * the scratch on `stream` and waits for that stream.  Make the first call
- * before any stream capture.  Completed calls leave the counters at zero;
+ * Every call looks up the scratch address with the current device (a
+ * failure returns Q4_ERR_CUDA).  The first call on each device -- and the
+ * first after the device's context was destroyed and created again, which
+ * gives the array a new address -- does setup: it zero-fills the scratch on
+ * `stream` and waits for that stream.  Make that call before any stream
+ * capture.  Completed calls leave the counters at zero;
  * after q4_sync_status has reported Q4_ERR_TIMEOUT the next call zero-fills
  * the scratch again on its stream before launching.
  *

@@ -566,26 +566,27 @@ static __device__ __align__(256) unsigned char g_q4_noalloc_scratch[kNoAllocScra
 
 namespace {
 
-// Scratch address on the current device `dev`, set up on first use: the
-// symbol address is looked up with `dev` current and the scratch zero-filled
-// on `st`, then `st` is waited for.
+// Scratch address on the current device `dev`.  The symbol's address is
+// looked up on every call (with `dev` current): when it differs from the
+// cached one -- the first call on the device, or a context that was torn down
+// and created again, whose module load zeroed a fresh array -- the scratch
+// is treated as new: zero-filled on `st`, and `st` waited for.
 q4_status noalloc_scratch(int dev, cudaStream_t st, void** out) {
     if (dev < 0 || dev >= kMaxDevices) return Q4_ERR_UNSUPPORTED;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_q4_noalloc_scratch) != cudaSuccess || p == nullptr)
+        return Q4_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_q4_noalloc_scratch) != cudaSuccess || p == nullptr)
-            return Q4_ERR_CUDA;
+    if (g_noalloc_ptr[dev] != p) {
         if (cudaMemsetAsync(p, 0, kNoAllocScratchBytes, st) != cudaSuccess) return Q4_ERR_CUDA;
         if (cudaStreamSynchronize(st) != cudaSuccess) return Q4_ERR_CUDA;
         g_noalloc_ptr[dev] = p;
         g_noalloc_reclear[dev] = false;
     } else if (g_noalloc_reclear[dev]) {
-        if (cudaMemsetAsync(g_noalloc_ptr[dev], 0, kNoAllocScratchBytes, st) != cudaSuccess)
-            return Q4_ERR_CUDA;
+        if (cudaMemsetAsync(p, 0, kNoAllocScratchBytes, st) != cudaSuccess) return Q4_ERR_CUDA;
         g_noalloc_reclear[dev] = false;
     }
-    *out = g_noalloc_ptr[dev];
+    *out = p;
     return Q4_OK;
 }
 

@@ -95,4 +95,43 @@ def test_noalloc_matches_workspace_entry_two_calls_in_a_row():
         setup_done = True
         for k, y in enumerate(ys):
             _within(y, y_ref, f"case {i} call {k}")
-        assert torch.equal(ys[0], ys[1]), f"case {i}: the two calls differ"
+            # the same kernel, plan and fix-up order as q4_gemv: bit for bit
+            assert torch.equal(y, y_ref), f"case {i} call {k}: differs from q4_gemv"
+
+
+
+@pytest.mark.gpu
+def test_noalloc_rezeroes_scratch_after_reported_timeout():
+    """After q4_sync_status reports Q4_ERR_TIMEOUT (a bounded wait that ran
+    out may leave stream-K counters set), the next call zero-fills the static
+    scratch before launching: two calls after a provoked timeout still match
+    q4_gemv bit for bit and allocate nothing.  The timeout comes from the
+    library's self-test kernel, a bounded wait on a barrier nothing arrives
+    on, which ends by itself after 2 ms."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from post_weight_quantization_group_b200 import build
+    build.build()
+    q4.load_library()
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    out, inn, g, B = 4096, 4096, 128, 1
+    w = q4.q4_quantize_pack(wl.normal_weight(out, inn, 500, device=dev), g, True)
+    x = wl.activations(B, inn, 501, device=dev)
+    y_ref = q4.q4_gemv(w, x)
+    y0 = torch.empty(B, out, dtype=torch.bfloat16, device=dev)
+    q4.q4_gemv_noalloc(w, x, y=y0)  # set up (or reuse) the scratch
+    assert q4.q4_sync_status() == q4.Q4_OK
+    assert torch.equal(y0, y_ref)
+    assert q4.q4_selftest_wait_timeout(2_000_000) == q4.Q4_OK
+    assert q4.q4_sync_status() == q4.Q4_ERR_TIMEOUT
+    ys = [torch.full((B, out), float("nan"), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info(dev)[0]
+    for y in ys:
+        q4.q4_gemv_noalloc(w, x, y=y)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info(dev)[0] == free_before, "q4_gemv_noalloc allocated device memory"
+    assert q4.q4_sync_status() == q4.Q4_OK
+    for k, y in enumerate(ys):
+        assert torch.equal(y, y_ref), f"call {k} after the timeout differs from q4_gemv"
