@@ -241,6 +241,31 @@ Q4_API q4_status q4_gemm_skinny(const q4_weight* w, const void* x, q4_dtype x_dt
                                 size_t workspace_bytes, q4_stream stream);
 
 /*
+ * Several products that share their activations -- the q, k and v
+ * projections of a decoder layer, or its gate and up projections -- in one
+ * call: y_i = x W_i^T for i < n, the products a decode step runs back to back
+ * on one activation (arganzheng.life section 二.1: the decode step streams
+ * every weight once; ybb.press section 一: the bottleneck is the HBM read).
+ *   ws  n quantized weights, 1 <= n <= Q4_GROUP_MAX, all with the same `in`,
+ *       group_size and symmetric flag (else Q4_ERR_SHAPE); each as in q4_gemv;
+ *   x   [B, in], 1 <= B <= 128;  ys[i]  [B, ws[i].out] of y_dtype, not
+ *       overlapping one another;
+ *   workspace  q4_workspace_bytes(out, in, B, group_size) bytes (the size does
+ *       not depend on `out` for B <= 8).
+ * For B <= 8 it is one launch of the q4_gemv kernel whose stream-K range runs
+ * over the products' row tiles one after another (at most 65536 tiles of 128
+ * rows in all, else Q4_ERR_SHAPE), so no product pays its own launch, ramp-up
+ * and tail.  The result is deterministic and within q4_gemv's tolerance; it
+ * may differ from q4_gemv's in the last bits, because the split of a row
+ * tile's K range between CTAs differs.  For B > 8 it runs q4_gemm_skinny once
+ * per product, in order.
+ */
+#define Q4_GROUP_MAX 4
+Q4_API q4_status q4_gemv_grouped(const q4_weight* ws, int32_t n, const void* x, q4_dtype x_dtype,
+                                 int64_t B, void* const* ys, q4_dtype y_dtype, void* workspace,
+                                 size_t workspace_bytes, q4_stream stream);
+
+/*
  * Size of the static device scratch that q4_gemv_noalloc uses (3 MiB): it
  * covers every shape q4_gemv accepts on a GPU with up to 176 SMs.
  */

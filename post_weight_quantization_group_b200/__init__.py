@@ -42,7 +42,7 @@ ABI_SYMBOLS = (
     "q4_workspace_bytes", "q4_gemv_noalloc", "q4_quantize_pack_clip", "q4_quantize_pack_perm",
     "q4_permute_activations", "q8_quantize_per_channel", "q8_dequant", "q8_workspace_bytes",
     "q8_gemv", "kv_quantize_int8", "kv_dequant_int8", "kv_quantize_int4", "kv_dequant_int4",
-    "mxfp4_quantize", "mxfp4_dequant", "nvfp4_quantize", "nvfp4_dequant",
+    "mxfp4_quantize", "mxfp4_dequant", "nvfp4_quantize", "nvfp4_dequant", "q4_gemv_grouped",
 )
 
 
@@ -94,6 +94,7 @@ def load_library(path: str = LIB_PATH):
     lib.q4_gemv.argtypes = [W, P, S, I64, P, S, P, ctypes.c_size_t, P]
     lib.q4_gemm_skinny.argtypes = [W, P, S, I64, P, S, P, ctypes.c_size_t, P]
     lib.q4_gemv_noalloc.argtypes = [W, P, S, I64, P, S, P]
+    lib.q4_gemv_grouped.argtypes = [W, I32, P, S, I64, ctypes.POINTER(P), S, P, ctypes.c_size_t, P]
     lib.q4_workspace_bytes.argtypes = [I64, I64, I64, I32]
     lib.q4_workspace_bytes.restype = ctypes.c_size_t
     lib.bf16_gemv_ref_bw.argtypes = [P, I64, I64, P, I64, P, P]
@@ -335,6 +336,34 @@ def q4_gemm_skinny(w: Q4Weight, x: torch.Tensor, y: torch.Tensor | None = None, 
                    workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """y = x W_hat^T for B <= 128."""
     return _product("q4_gemm_skinny", w, x, y, y_dtype, workspace, stream)
+
+
+Q4_GROUP_MAX = 4
+
+
+def q4_gemv_grouped(ws, x: torch.Tensor, ys=None, y_dtype=None,
+                    workspace: torch.Tensor | None = None, stream=None):
+    """[y_i = x W_hat_i^T for W_i in ws] in one call (weights sharing ``in``,
+    group size and symmetry; at most Q4_GROUP_MAX); B <= 8 is one launch."""
+    lib = load_library()
+    if x.dim() != 2:
+        raise ValueError("x must be [B, in]")
+    ws = list(ws)
+    B = x.shape[0]
+    if ys is None:
+        ys = [torch.empty(B, w.out, dtype=y_dtype or x.dtype, device=x.device) for w in ws]
+    ys = list(ys)
+    if len(ys) != len(ws):
+        raise ValueError("one output per weight")
+    if workspace is None:
+        workspace = workspace_for(ws[0], B, x.device)
+    arr = (_CWeight * len(ws))(*[w.c_struct() for w in ws])
+    yp = (ctypes.c_void_p * len(ys))(*[_ptr(y) for y in ys])
+    st = lib.q4_gemv_grouped(arr, len(ws), _ptr(x), _DT[x.dtype], B, yp, _DT[ys[0].dtype],
+                             _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _stream(stream))
+    _check(st, "q4_gemv_grouped")
+    return ys
 
 
 def q4_gemv_noalloc(w: Q4Weight, x: torch.Tensor, y: torch.Tensor | None = None, y_dtype=None,

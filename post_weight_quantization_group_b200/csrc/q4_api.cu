@@ -279,6 +279,7 @@ constexpr int kGemvRT = kGemvCW * kGemvMT * 16;
 #define Q4_SK_CW 8
 #endif
 constexpr int kSkCW = Q4_SK_CW;
+static_assert(Q4_GROUP_MAX == kSkMaxGroup, "group size of the ABI and the kernel");
 constexpr int kSkRT = kSkCW * 16;
 constexpr int kSkCtasPerSm = 2;
 constexpr int kSkMinIters = 2;
@@ -331,11 +332,24 @@ SkPlan product_plan(int64_t out, int64_t in, int64_t B, int sms) {
     return B <= 8 ? sk_plan(out, in, sms) : tc_plan(out, in, B, sms);
 }
 
+// One launch over n products that share x (same in, group size, symmetry):
+// their row tiles are concatenated into one stream-K iteration space.
 template <bool BF16, int GS, bool SYM>
-q4_status run_gemv(const q4_weight* w, const void* x, int64_t B, void* y, int ydt, void* ws,
-                   size_t ws_bytes, cudaStream_t st) {
+q4_status run_gemv(const q4_weight* const* wv, int n, const void* x, int64_t B, void* const* ys,
+                   int ydt, void* ws, size_t ws_bytes, cudaStream_t st) {
     const int dev = current_device();
-    const SkPlan p = sk_plan(w->out, w->in, sm_count(dev));
+    SkGroup grp;
+    std::memset(&grp, 0, sizeof(grp));
+    grp.n = n;
+    int64_t tiles = 0;
+    for (int i = 0; i < n; ++i) {
+        grp.tile_beg[i] = tiles;
+        tiles += (wv[i]->out + kSkRT - 1) / kSkRT;
+    }
+    grp.tile_beg[n] = tiles;
+    if (tiles > 65536) return Q4_ERR_SHAPE;  // one workspace counter per row tile
+    const int64_t in = wv[0]->in;
+    const SkPlan p = sk_plan(tiles * kSkRT, in, sm_count(dev));
     if (!ws || ws_bytes < p.ws_bytes) return Q4_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return Q4_ERR_ALIGNMENT;
     // Deepest ring that still lets two CTAs share an SM.  From B = 4 on, two
@@ -351,31 +365,38 @@ q4_status run_gemv(const q4_weight* w, const void* x, int64_t B, void* y, int yd
     const bool two_helpers = B >= 4;
     if (two_helpers && (stages & 1)) geo = sk_geom(kSkRT, --stages, static_cast<int>(B), SYM);
     const int helpers = two_helpers ? 2 : 1;
-    const int64_t G = w->in / GS;
-    // scale / zero windows by TMA when their rows are 16-byte aligned
-    const bool meta_tma = (G % 8) == 0 && aligned(w->scales, 16) && (SYM || aligned(w->zeros, 16));
-    CUtensorMap tmap_w, tmap_x, tmap_s, tmap_z;
-    std::memset(&tmap_s, 0, sizeof(tmap_s));
-    std::memset(&tmap_z, 0, sizeof(tmap_z));
-    if (!make_tmap_2d(&tmap_w, w->qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
-                      static_cast<uint64_t>(w->out), static_cast<uint64_t>(w->in / 2), kSkRT,
-                      kChunkBytes))
-        return Q4_ERR_CUDA;
+    const int64_t G = in / GS;
+    // scale / zero windows by TMA when every product's rows are 16-byte aligned
+    bool meta_tma = (G % 8) == 0;
+    for (int i = 0; i < n; ++i)
+        meta_tma = meta_tma && aligned(wv[i]->scales, 16) && (SYM || aligned(wv[i]->zeros, 16));
+    for (int i = 0; i < n; ++i) {
+        const q4_weight* w = wv[i];
+        grp.scales[i] = reinterpret_cast<const uint16_t*>(w->scales);
+        grp.zeros[i] = reinterpret_cast<const uint16_t*>(w->zeros);
+        grp.y[i] = ys[i];
+        grp.out[i] = w->out;
+        if (!make_tmap_2d(&grp.w[i], w->qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                          static_cast<uint64_t>(w->out), static_cast<uint64_t>(in / 2), kSkRT,
+                          kChunkBytes))
+            return Q4_ERR_CUDA;
+        if (meta_tma) {
+            if (!make_tmap_2d(&grp.s[i], w->scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                              static_cast<uint64_t>(w->out), static_cast<uint64_t>(G), kSkRT, 8,
+                              CU_TENSOR_MAP_SWIZZLE_NONE))
+                return Q4_ERR_CUDA;
+            if (!SYM && !make_tmap_2d(&grp.z[i], w->zeros, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                                      static_cast<uint64_t>(w->out), static_cast<uint64_t>(G),
+                                      kSkRT, 8, CU_TENSOR_MAP_SWIZZLE_NONE))
+                return Q4_ERR_CUDA;
+        }
+    }
+    CUtensorMap tmap_x;
     if (!make_tmap_2d(&tmap_x, x,
                       BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                      static_cast<uint64_t>(B), static_cast<uint64_t>(w->in),
+                      static_cast<uint64_t>(B), static_cast<uint64_t>(in),
                       static_cast<uint32_t>(B), kChunkCodes, CU_TENSOR_MAP_SWIZZLE_NONE))
         return Q4_ERR_CUDA;
-    if (meta_tma) {
-        if (!make_tmap_2d(&tmap_s, w->scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                          static_cast<uint64_t>(w->out), static_cast<uint64_t>(G), kSkRT, 8,
-                          CU_TENSOR_MAP_SWIZZLE_NONE))
-            return Q4_ERR_CUDA;
-        if (!SYM && !make_tmap_2d(&tmap_z, w->zeros, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                                  static_cast<uint64_t>(w->out), static_cast<uint64_t>(G), kSkRT,
-                                  8, CU_TENSOR_MAP_SWIZZLE_NONE))
-            return Q4_ERR_CUDA;
-    }
     auto kernel = two_helpers ? q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 2>
                               : q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 1>;
     if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), false)) return Q4_ERR_CUDA;
@@ -385,26 +406,31 @@ q4_status run_gemv(const q4_weight* w, const void* x, int64_t B, void* y, int yd
     unsigned* ws_count = reinterpret_cast<unsigned*>(ws);
     float* ws_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kWsCounterBytes);
     return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3((kSkCW + 1 + helpers) * 32),
-                          geo.total, 1, true, st, tmap_w, tmap_x, tmap_s, tmap_z, meta_tma ? 1 : 0,
-                          reinterpret_cast<const uint16_t*>(w->scales),
-                          reinterpret_cast<const uint16_t*>(w->zeros), stages,
-                          static_cast<int>(B), w->out, w->in, p.nchunks, p.T, y, ydt, ws_part,
-                          ws_count, status);
+                     geo.total, 1, true, st, grp, tmap_x, meta_tma ? 1 : 0, stages,
+                     static_cast<int>(B), in, p.nchunks, p.T, ydt, ws_part, ws_count, status);
+}
+
+template <bool BF16>
+q4_status dispatch_gemv(const q4_weight* const* wv, int n, const void* x, int64_t B,
+                        void* const* ys, int ydt, void* ws, size_t wsb, cudaStream_t st) {
+    const bool sym = wv[0]->symmetric != 0;
+    switch (wv[0]->group_size) {
+        case 32: return sym ? run_gemv<BF16, 32, true>(wv, n, x, B, ys, ydt, ws, wsb, st)
+                            : run_gemv<BF16, 32, false>(wv, n, x, B, ys, ydt, ws, wsb, st);
+        case 64: return sym ? run_gemv<BF16, 64, true>(wv, n, x, B, ys, ydt, ws, wsb, st)
+                            : run_gemv<BF16, 64, false>(wv, n, x, B, ys, ydt, ws, wsb, st);
+        case 128: return sym ? run_gemv<BF16, 128, true>(wv, n, x, B, ys, ydt, ws, wsb, st)
+                             : run_gemv<BF16, 128, false>(wv, n, x, B, ys, ydt, ws, wsb, st);
+        default: return Q4_ERR_UNSUPPORTED;
+    }
 }
 
 template <bool BF16>
 q4_status dispatch_gemv(const q4_weight* w, const void* x, int64_t B, void* y, int ydt, void* ws,
                         size_t wsb, cudaStream_t st) {
-    const bool sym = w->symmetric != 0;
-    switch (w->group_size) {
-        case 32: return sym ? run_gemv<BF16, 32, true>(w, x, B, y, ydt, ws, wsb, st)
-                            : run_gemv<BF16, 32, false>(w, x, B, y, ydt, ws, wsb, st);
-        case 64: return sym ? run_gemv<BF16, 64, true>(w, x, B, y, ydt, ws, wsb, st)
-                            : run_gemv<BF16, 64, false>(w, x, B, y, ydt, ws, wsb, st);
-        case 128: return sym ? run_gemv<BF16, 128, true>(w, x, B, y, ydt, ws, wsb, st)
-                             : run_gemv<BF16, 128, false>(w, x, B, y, ydt, ws, wsb, st);
-        default: return Q4_ERR_UNSUPPORTED;
-    }
+    const q4_weight* wv[1] = {w};
+    void* ys[1] = {y};
+    return dispatch_gemv<BF16>(wv, 1, x, B, ys, ydt, ws, wsb, st);
 }
 
 // ------------------------------------------- W8A16 (per-channel INT8)
@@ -828,6 +854,44 @@ q4_status q4_gemm_skinny(const q4_weight* w, const void* x, q4_dtype x_dtype, in
     return x_dtype == Q4_BF16
                ? dispatch_skinny<true>(w, x, B, y, ydt, workspace, workspace_bytes, st)
                : dispatch_skinny<false>(w, x, B, y, ydt, workspace, workspace_bytes, st);
+}
+
+q4_status q4_gemv_grouped(const q4_weight* ws, int32_t n, const void* x, q4_dtype x_dtype,
+                          int64_t B, void* const* ys, q4_dtype y_dtype, void* workspace,
+                          size_t workspace_bytes, q4_stream stream) {
+    if (!ws || !ys || n < 1 || n > Q4_GROUP_MAX) return Q4_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {
+        q4_status s = validate_product(&ws[i], x, x_dtype, B, ys[i], y_dtype, 128);
+        if (s != Q4_OK) return s;
+        if (ws[i].in != ws[0].in || ws[i].group_size != ws[0].group_size ||
+            ws[i].symmetric != ws[0].symmetric)
+            return Q4_ERR_SHAPE;
+    }
+    if (B > 8) {
+        // the tensor-core kernel runs one product per launch
+        for (int i = 0; i < n; ++i) {
+            q4_status s = q4_gemm_skinny(&ws[i], x, x_dtype, B, ys[i], y_dtype, workspace,
+                                         workspace_bytes, stream);
+            if (s != Q4_OK) return s;
+        }
+        return Q4_OK;
+    }
+    const q4_weight* wv[Q4_GROUP_MAX];
+    void* yv[Q4_GROUP_MAX];
+    int m = 0;
+    for (int i = 0; i < n; ++i) {
+        if (ws[i].out == 0) continue;  // nothing to read or write
+        wv[m] = &ws[i];
+        yv[m] = ys[i];
+        ++m;
+    }
+    if (m == 0) return Q4_OK;
+    if (!workspace) return Q4_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int ydt = y_dtype == Q4_F32 ? 2 : (y_dtype == Q4_BF16 ? 1 : 0);
+    return x_dtype == Q4_BF16
+               ? dispatch_gemv<true>(wv, m, x, B, yv, ydt, workspace, workspace_bytes, st)
+               : dispatch_gemv<false>(wv, m, x, B, yv, ydt, workspace, workspace_bytes, st);
 }
 
 q4_status q4_gemv_noalloc(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B,

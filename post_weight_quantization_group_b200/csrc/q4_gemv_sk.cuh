@@ -56,6 +56,29 @@ namespace q4dev {
 
 constexpr int kSkMaxStages = 4;
 
+// Up to kSkMaxGroup products that share their activations (one call covers,
+// e.g., the q, k and v projections of a layer): their row tiles are
+// concatenated into one stream-K iteration space, product i owning the global
+// row tiles [tile_beg[i], tile_beg[i + 1]).
+constexpr int kSkMaxGroup = 4;
+struct SkGroup {
+    CUtensorMap w[kSkMaxGroup], s[kSkMaxGroup], z[kSkMaxGroup];
+    const uint16_t* scales[kSkMaxGroup];
+    const uint16_t* zeros[kSkMaxGroup];
+    void* y[kSkMaxGroup];
+    int64_t out[kSkMaxGroup];
+    int64_t tile_beg[kSkMaxGroup + 1];
+    int n;
+};
+
+// Product that owns global row tile `tile`.
+__device__ __forceinline__ int sk_product(const SkGroup& g, int64_t tile) {
+    int i = 0;
+#pragma unroll
+    for (int k = 1; k < kSkMaxGroup; ++k) i += (k < g.n && tile >= g.tile_beg[k]) ? 1 : 0;
+    return i;
+}
+
 struct SkGeom {
     size_t w_bytes, off_m, m_bytes;              // weight tiles, per-stage slots
     size_t off_x, off_xp, off_sx, off_sc, off_zc;  // inside a per-stage slot
@@ -106,13 +129,9 @@ __device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v
 // budget of its own block size.
 template <bool BF16, int GS, bool SYM, int CW, int NH>
 __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
-    q4_gemv_sk_kernel(const __grid_constant__ CUtensorMap tmap_w,
-                      const __grid_constant__ CUtensorMap tmap_x,
-                      const __grid_constant__ CUtensorMap tmap_s,
-                      const __grid_constant__ CUtensorMap tmap_z, int meta_tma,
-                      const uint16_t* __restrict__ scales, const uint16_t* __restrict__ zeros,
-                      int stages, int B, int64_t out, int64_t in, int nchunks, int64_t T,
-                      void* __restrict__ y, int ydt, float* __restrict__ ws_part,
+    q4_gemv_sk_kernel(const __grid_constant__ SkGroup grp,
+                      const __grid_constant__ CUtensorMap tmap_x, int meta_tma, int stages, int B,
+                      int64_t in, int nchunks, int64_t T, int ydt, float* __restrict__ ws_part,
                       unsigned* __restrict__ ws_count, unsigned* __restrict__ status) {
     constexpr int RT = CW * 16;
     constexpr int GPC = kChunkCodes / GS;  // groups per chunk
@@ -155,7 +174,7 @@ __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
     if (warp == CW) {
         // ------------------------------------------------------ producer
         if (lane == 0 && nit > 0) {
-            prefetch_tmap(&tmap_w);
+            for (int i = 0; i < grp.n; ++i) prefetch_tmap(&grp.w[i]);
             prefetch_tmap(&tmap_x);
             const uint32_t tx = RT * kChunkBytes + B * 512 +
                                 (meta_tma ? RT * 16 * (SYM ? 1 : 2) : 0);
@@ -166,11 +185,13 @@ __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
                 for (int c = 0; c < pre; ++c) {
                     uint8_t* ms = smem + geo.off_m + geo.m_bytes * c;
                     mbar_arrive_expect_tx(&full[c], tx);
-                    tma_load_2d(smem + geo.w_bytes * c, &tmap_w, chunk * kChunkBytes, tile * RT, &full[c]);
+                    const int pi = sk_product(grp, tile);
+                    const int lt = static_cast<int>(tile - grp.tile_beg[pi]);
+                    tma_load_2d(smem + geo.w_bytes * c, &grp.w[pi], chunk * kChunkBytes, lt * RT, &full[c]);
                     if (meta_tma) {
                         const int win = (chunk * GPC) & ~7;
-                        tma_load_2d(ms + geo.off_sc, &tmap_s, win, tile * RT, &full[c]);
-                        if constexpr (!SYM) tma_load_2d(ms + geo.off_zc, &tmap_z, win, tile * RT, &full[c]);
+                        tma_load_2d(ms + geo.off_sc, &grp.s[pi], win, lt * RT, &full[c]);
+                        if constexpr (!SYM) tma_load_2d(ms + geo.off_zc, &grp.z[pi], win, lt * RT, &full[c]);
                     }
                     if (++chunk == nchunks) {
                         chunk = 0;
@@ -188,11 +209,13 @@ __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
                 uint8_t* ms = smem + geo.off_m + geo.m_bytes * s;
                 if (c >= pre) {
                     mbar_arrive_expect_tx(&full[s], tx);
-                    tma_load_2d(smem + geo.w_bytes * s, &tmap_w, chunk * kChunkBytes, tile * RT, &full[s]);
+                    const int pi = sk_product(grp, tile);
+                    const int lt = static_cast<int>(tile - grp.tile_beg[pi]);
+                    tma_load_2d(smem + geo.w_bytes * s, &grp.w[pi], chunk * kChunkBytes, lt * RT, &full[s]);
                     if (meta_tma) {
                         const int win = (chunk * GPC) & ~7;
-                        tma_load_2d(ms + geo.off_sc, &tmap_s, win, tile * RT, &full[s]);
-                        if constexpr (!SYM) tma_load_2d(ms + geo.off_zc, &tmap_z, win, tile * RT, &full[s]);
+                        tma_load_2d(ms + geo.off_sc, &grp.s[pi], win, lt * RT, &full[s]);
+                        if constexpr (!SYM) tma_load_2d(ms + geo.off_zc, &grp.z[pi], win, lt * RT, &full[s]);
                     }
                 }
                 tma_load_2d(ms + geo.off_x, &tmap_x, chunk * kChunkCodes, 0, &full[s]);
@@ -300,11 +323,16 @@ __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
                 uint16_t* zcs = reinterpret_cast<uint16_t*>(st + geo.off_zc);
                 const int64_t g0 = static_cast<int64_t>(chunk) * GPC;
                 const int wofs = (chunk * GPC) & 7;
+                const int pi = sk_product(grp, tile);
+                const int64_t out_p = grp.out[pi];
+                const uint16_t* scales = grp.scales[pi];
+                const uint16_t* zeros = grp.zeros[pi];
+                const int64_t row_p = (static_cast<int64_t>(tile) - grp.tile_beg[pi]) * RT;
                 for (int idx = lane; idx < RT * GPC; idx += 32) {
                     const int r = idx / GPC;
                     const int gq = idx % GPC;
-                    const int64_t row = static_cast<int64_t>(tile) * RT + r;
-                    const bool okg = row < out && g0 + gq < G;
+                    const int64_t row = row_p + r;
+                    const bool okg = row < out_p && g0 + gq < G;
                     scs[r * 8 + wofs + gq] = okg ? __ldg(scales + row * G + g0 + gq) : 0;
                     if constexpr (!SYM) zcs[r * 8 + wofs + gq] = okg ? __ldg(zeros + row * G + g0 + gq) : 0;
                 }
@@ -432,7 +460,10 @@ __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
         // ---------------------------------------------- segment epilogue
         if (cur_chunk == nchunks - 1 || c == nit - 1) {
             const int64_t tile = cur_tile;
-            const int64_t row0 = tile * RT;
+            const int pi = sk_product(grp, tile);
+            const int64_t out = grp.out[pi];
+            void* const y = grp.y[pi];
+            const int64_t row0 = (tile - grp.tile_beg[pi]) * RT;
             const bool whole = (c - seg_start) == cur_chunk && cur_chunk == nchunks - 1;
             if (whole) {
 #pragma unroll
