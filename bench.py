@@ -67,6 +67,13 @@ def dense_bytes(out, inn, B):
     return out * inn * 2 + B * inn * 2 + B * out * 2
 
 
+def fp4_bytes(out, inn, fmt, B):
+    """Algorithmic bytes of one W4A4 product: FP4 codes and scale bytes of W
+    and x, y in bf16 (the NVFP4 tensor scales are 8 bytes and left out)."""
+    blk = 32 if fmt == "mxfp4" else 16
+    return (out + B) * (inn // 2 + inn // blk) + B * out * 2
+
+
 def quant_bytes(out, inn, g, sym=True):
     return out * inn * 2 + out * inn // 2 + out * (inn // g) * 2 * (1 if sym else 2)
 
@@ -787,7 +794,9 @@ def run_op(args):
     ``w8a16-70b`` = q8_gemv on the Llama-3-70B down_proj (8192 x 28672, batch
     --batch, two weight copies rotating); ``q4-70b-down`` = q4_gemm_skinny
     (sym g128) on the same shape and batch (the B <= 8 kernel or, above, the
-    tcgen05 kernel); ``kv8-70b-32k`` = kv_quantize_int8
+    tcgen05 kernel); ``nvfp4-70b-down`` / ``mxfp4-70b-down`` = fp4_gemm (W4A4,
+    seeded FP4 weight bytes, activations quantized by the library) on the same
+    shape and batch; ``kv8-70b-32k`` = kv_quantize_int8
     of one layer's K cache at 32768 tokens ([1, 8, 32768, 128] bf16, four
     caches rotating).  Prints one JSON line (CUDA-event time per call)."""
     import torch
@@ -826,6 +835,24 @@ def run_op(args):
         fn = lambda: q4.q4_gemm_skinny(ws[next(it) % 2], x, y=y, workspace=wsp)
         nbytes = algo_bytes(out, inn, 128, B)
         name, cfg = "W4A16 INT4 product (sym g128)", {"workload": f"Llama-3-70B down_proj {out}x{inn}", "batch": B}
+    elif args.workload in ("nvfp4-70b-down", "mxfp4-70b-down"):
+        fmt = args.workload.split("-")[0]
+        out, inn = wl.LLAMA3_70B["down_proj"]
+        B = args.batch
+        ws = []
+        for i in range(2):
+            p, s = wl.fp4_operand(out, inn, fmt, 40 + i)
+            ts = (torch.tensor([wl.FP4_W_TENSOR_SCALE], dtype=torch.float32, device=device)
+                  if fmt == "nvfp4" else None)
+            ws.append(q4.FP4Weight(p.to(device), s.to(device), out, inn, fmt, ts))
+        X = q4.fp4_quantize(wl.activations(B, inn, 31, device=device), fmt)
+        y = torch.empty(B, out, dtype=torch.bfloat16, device=device)
+        wsp = q4.fp4_workspace_for(ws[0], B, device)
+        it = iter(range(1 << 30))
+        fn = lambda: q4.fp4_gemm(ws[next(it) % 2], X, y=y, workspace=wsp)
+        nbytes = fp4_bytes(out, inn, fmt, B)
+        name, cfg = (f"W4A4 {fmt.upper()} product (block-scaled tcgen05)",
+                     {"workload": f"Llama-3-70B down_proj {out}x{inn}", "batch": B})
     else:
         shape = (1, wl.LLAMA3_70B_KV_HEADS, 32768, wl.LLAMA3_70B_HEAD_DIM)
         caches = [wl.kv_cache(*shape, seed=70 + i, dtype=torch.bfloat16, device=device) for i in range(4)]
@@ -856,7 +883,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama3-8b",
                     choices=["llama3-8b", "llama3-70b-stack", "w8a16-70b", "q4-70b-down",
-                             "kv8-70b-32k"])
+                             "kv8-70b-32k", "nvfp4-70b-down", "mxfp4-70b-down"])
     ap.add_argument("--batch", type=int, default=1, help="batch of the llama3-70b-stack workload")
     ap.add_argument("--layers", type=int, default=32,
                     help="distinct decoder layers per step (32 = the Llama-3-8B depth)")
@@ -871,7 +898,8 @@ def main():
         run_reference(args)
     elif args.workload == "llama3-70b-stack":
         run_stack(args)
-    elif args.workload in ("w8a16-70b", "q4-70b-down", "kv8-70b-32k"):
+    elif args.workload in ("w8a16-70b", "q4-70b-down", "kv8-70b-32k", "nvfp4-70b-down",
+                           "mxfp4-70b-down"):
         run_op(args)
     else:
         run_ours(args)

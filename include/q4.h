@@ -406,6 +406,47 @@ Q4_API q4_status nvfp4_dequant(const uint8_t* packed, const uint8_t* scales,
                                const float* tensor_scale, int64_t out, int64_t in, void* W_hat,
                                q4_dtype out_dtype, q4_stream stream);
 
+/* W4A4 product of two FP4 operands of the same format on the block-scaled
+ * tensor cores ("post-training-quantization-gptq-awq-and-rotation"
+ * (arganzheng.life), section 九.2: Blackwell multiplies microscaled FP4
+ * operands natively, the block scales applied inside the MMA):
+ *
+ *   y[b, r] = g * sum_k e2m1(wq[r, k]) * S_w[r, k / VS] * e2m1(xq[b, k]) * S_x[b, k / VS]
+ *
+ *   MXFP4 (format Q4_FP4_MXFP4): VS = 32, S = 2^(byte - 127), g = 1;
+ *   NVFP4 (format Q4_FP4_NVFP4): VS = 16, S = e4m3(byte),
+ *                                g = w_tensor_scale * x_tensor_scale.
+ *
+ * Both operands are laid out as mxfp4_quantize / nvfp4_quantize write them
+ * (the activations are quantized as a [B, in] matrix by the same calls):
+ *   w_packed        [out, in/2] codes, 16-byte aligned
+ *   w_scales        [out, in/VS] scale bytes, 16-byte aligned
+ *   w_tensor_scale  one fp32 on the device (NVFP4; ignored for MXFP4)
+ *   x_packed        [B, in/2] codes, 16-byte aligned
+ *   x_scales        [B, in/VS] scale bytes, 16-byte aligned
+ *   x_tensor_scale  one fp32 on the device (NVFP4; ignored for MXFP4)
+ *   y               [B, out] in y_dtype (f16, bf16 or f32), written
+ *   in              a multiple of 256 (NVFP4) or 512 (MXFP4): the scale rows
+ *                   are read by TMA, whose row strides are multiples of 16 B
+ *   workspace       at least fp4_gemm_workspace_bytes(format, out, in, B)
+ *                   bytes, 256-byte aligned, zero-filled once before its
+ *                   first use (the kernels leave it zeroed again); one call
+ *                   at a time per workspace
+ * Accumulation is fp32 inside the tensor core; the result is deterministic
+ * (split tiles add their partials in a fixed order).  B > 128 runs as slices
+ * of 128 activation rows.  Errors: Q4_ERR_INVALID_ARG (format, dtype, null
+ * pointer), Q4_ERR_SHAPE, Q4_ERR_ALIGNMENT, Q4_ERR_WORKSPACE; a device-side
+ * wait that runs out sets Q4_ERR_TIMEOUT for q4_sync_status.
+ */
+#define Q4_FP4_MXFP4 0
+#define Q4_FP4_NVFP4 1
+Q4_API size_t fp4_gemm_workspace_bytes(int32_t format, int64_t out, int64_t in, int64_t B);
+Q4_API q4_status fp4_gemm(int32_t format, const uint8_t* w_packed, const uint8_t* w_scales,
+                          const float* w_tensor_scale, int64_t out, int64_t in,
+                          const uint8_t* x_packed, const uint8_t* x_scales,
+                          const float* x_tensor_scale, int64_t B, void* y, q4_dtype y_dtype,
+                          void* workspace, size_t workspace_bytes, q4_stream stream);
+
 /* --------------------------------------------------------------- KV cache
  *
  * A KV cache [batch, heads, seq, head_dim] in fp16 or bf16 is passed as

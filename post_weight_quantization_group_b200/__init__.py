@@ -43,6 +43,7 @@ ABI_SYMBOLS = (
     "q4_permute_activations", "q8_quantize_per_channel", "q8_dequant", "q8_workspace_bytes",
     "q8_gemv", "kv_quantize_int8", "kv_dequant_int8", "kv_quantize_int4", "kv_dequant_int4",
     "mxfp4_quantize", "mxfp4_dequant", "nvfp4_quantize", "nvfp4_dequant", "q4_gemv_grouped",
+    "fp4_gemm_workspace_bytes", "fp4_gemm",
 )
 
 
@@ -113,13 +114,16 @@ def load_library(path: str = LIB_PATH):
     lib.mxfp4_dequant.argtypes = [P, P, I64, I64, P, S, P]
     lib.nvfp4_quantize.argtypes = [P, S, I64, I64, P, P, P, P]
     lib.nvfp4_dequant.argtypes = [P, P, P, I64, I64, P, S, P]
+    lib.fp4_gemm_workspace_bytes.argtypes = [I32, I64, I64, I64]
+    lib.fp4_gemm_workspace_bytes.restype = ctypes.c_size_t
+    lib.fp4_gemm.argtypes = [I32, P, P, P, I64, I64, P, P, P, I64, P, S, P, ctypes.c_size_t, P]
     for f in ("q4_quantize_pack", "q4_quantize_pack_clip", "q4_quantize_pack_perm",
               "q4_permute_activations", "q4_dequant", "q4_gemv",
               "q4_gemm_skinny", "q4_gemv_noalloc",
               "bf16_gemv_ref_bw", "q4_sync_status", "q4_selftest_wait_timeout",
               "q8_quantize_per_channel", "q8_dequant", "q8_gemv", "kv_quantize_int8",
               "kv_dequant_int8", "kv_quantize_int4", "kv_dequant_int4", "mxfp4_quantize",
-              "mxfp4_dequant", "nvfp4_quantize", "nvfp4_dequant"):
+              "mxfp4_dequant", "nvfp4_quantize", "nvfp4_dequant", "fp4_gemm"):
         getattr(lib, f).restype = S
     lib.q4_status_string.argtypes = [S]
     lib.q4_status_string.restype = ctypes.c_char_p
@@ -605,3 +609,44 @@ def fp4_dequant(w: FP4Weight, out_dtype=torch.float32, W_hat: torch.Tensor | Non
                                w.in_features, _ptr(W_hat), _DT[W_hat.dtype], _stream(stream))
     _check(st, f"{w.fmt}_dequant")
     return W_hat
+
+
+FP4_FORMATS = {"mxfp4": 0, "nvfp4": 1}  # Q4_FP4_MXFP4, Q4_FP4_NVFP4
+
+
+def fp4_quantize(W: torch.Tensor, fmt: str, stream=None) -> FP4Weight:
+    """mxfp4_quantize or nvfp4_quantize by name; activations [B, in] are
+    quantized the same way as weights [out, in]."""
+    if fmt == "mxfp4":
+        return mxfp4_quantize(W, stream)
+    if fmt == "nvfp4":
+        return nvfp4_quantize(W, stream)
+    raise ValueError(f"unknown FP4 format {fmt!r}")
+
+
+def fp4_workspace_for(w: FP4Weight, B: int, device) -> torch.Tensor:
+    need = int(load_library().fp4_gemm_workspace_bytes(FP4_FORMATS[w.fmt], w.out, w.in_features, B))
+    return _shared_workspace(need, device)
+
+
+def fp4_gemm(w: FP4Weight, x: FP4Weight, y: torch.Tensor | None = None,
+             y_dtype=torch.bfloat16, workspace: torch.Tensor | None = None,
+             stream=None) -> torch.Tensor:
+    """W4A4 product y [B, out] of FP4 weights ``w`` [out, in] and FP4
+    activations ``x`` [B, in] of the same format, on the block-scaled tensor
+    cores (the C entry point fp4_gemm)."""
+    lib = load_library()
+    if w.fmt != x.fmt or w.in_features != x.in_features:
+        raise ValueError("w and x must share the FP4 format and `in`")
+    B = x.out
+    dev = w.packed.device
+    if y is None:
+        y = torch.empty(B, w.out, dtype=y_dtype, device=dev)
+    if workspace is None:
+        workspace = fp4_workspace_for(w, B, dev)
+    st = lib.fp4_gemm(FP4_FORMATS[w.fmt], _ptr(w.packed), _ptr(w.scales), _ptr(w.tensor_scale),
+                      w.out, w.in_features, _ptr(x.packed), _ptr(x.scales), _ptr(x.tensor_scale),
+                      B, _ptr(y), _DT[y.dtype], _ptr(workspace),
+                      workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "fp4_gemm")
+    return y

@@ -1,7 +1,7 @@
 // q4_api.cu -- the C ABI of include/q4.h: argument validation, launch
 // planning, TMA descriptor encoding and kernel launches.  All kernels live in
 // this translation unit (q4_quant.cuh, q4_gemv.cuh, q4_gemv_sk.cuh,
-// q4_skinny_tc.cuh, q8_gemv.cuh, q8_quant.cuh, fp4_quant.cuh).
+// q4_skinny_tc.cuh, q8_gemv.cuh, q8_quant.cuh, fp4_quant.cuh, fp4_gemm.cuh).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -21,6 +21,7 @@
 #include "q8_gemv.cuh"
 #include "q8_quant.cuh"
 #include "fp4_quant.cuh"
+#include "fp4_gemm.cuh"
 
 namespace {
 
@@ -661,6 +662,68 @@ q4_status fp4_dequant(const uint8_t* packed, const uint8_t* scales, const float*
             pw, scales, tensor_scale, nwords, reinterpret_cast<__nv_bfloat16*>(W_hat));
     return launch_status(cudaSuccess);
 }
+
+// ------------------------------------------- FP4 block-scaled product
+constexpr int kF4MinIters = 4;
+constexpr int64_t kF4MaxB = 128;  // activation rows per launch (the MMA's N)
+
+int f4_nt(int64_t B) { return B <= 16 ? 16 : B <= 32 ? 32 : B <= 64 ? 64 : 128; }
+
+SkPlan fp4_plan(int64_t out, int64_t in, int64_t B, int sms) {
+    return stream_k_plan(out, in, kF4RT, sms, kF4MinIters, f4_nt(B), kF4ChunkCodes);
+}
+
+template <bool NV, int NT>
+q4_status run_fp4(const uint8_t* wq, const uint8_t* wsc, const float* wts, int64_t out,
+                  int64_t in, const uint8_t* xq, const uint8_t* xsc, const float* xts, int64_t B,
+                  void* y, int ydt, void* ws, size_t ws_bytes, cudaStream_t st) {
+    constexpr int VS = F4Fmt<NV>::VS;
+    constexpr int SFB = F4Fmt<NV>::sf_bytes;
+    const int dev = current_device();
+    const SkPlan p = fp4_plan(out, in, B, sm_count(dev));
+    if (p.row_tiles > static_cast<int64_t>(kWsCounterBytes / 4)) return Q4_ERR_SHAPE;
+    if (!ws || ws_bytes < p.ws_bytes) return Q4_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return Q4_ERR_ALIGNMENT;
+    const size_t smax = static_cast<size_t>(max_smem_optin(dev));
+    int stages = kF4MaxStages;
+    F4Geom geo = f4_geom(NT, SFB, stages);
+    while (stages > 2 && geo.total > smax) geo = f4_geom(NT, SFB, --stages);
+    if (geo.total > smax) return Q4_ERR_UNSUPPORTED;
+    CUtensorMap tmap_w, tmap_sw, tmap_x, tmap_sx;
+    const uint64_t cb = static_cast<uint64_t>(in / 2), sb = static_cast<uint64_t>(in / VS);
+    if (!make_tmap_2d(&tmap_w, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(out),
+                      cb, kF4RT, kF4Box) ||
+        !make_tmap_2d(&tmap_sw, wsc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                      static_cast<uint64_t>(out), sb, kF4RT, SFB, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_tmap_2d(&tmap_x, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(B), cb,
+                      NT, kF4Box) ||
+        !make_tmap_2d(&tmap_sx, xsc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(B),
+                      sb, NT, SFB, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return Q4_ERR_CUDA;
+    auto kernel = fp4_gemm_tc_kernel<NV, NT>;
+    if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), false)) return Q4_ERR_CUDA;
+    unsigned* status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
+        return Q4_ERR_CUDA;
+    unsigned* ws_count = reinterpret_cast<unsigned*>(ws);
+    float* ws_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kWsCounterBytes);
+    return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3(kF4Threads), geo.total, 1,
+                     true, st, tmap_w, tmap_sw, tmap_x, tmap_sx, wts, xts, stages,
+                     static_cast<int>(B), out, p.nchunks, p.T, y, ydt, ws_part, ws_count, status);
+}
+
+template <bool NV>
+q4_status dispatch_fp4(const uint8_t* wq, const uint8_t* wsc, const float* wts, int64_t out,
+                       int64_t in, const uint8_t* xq, const uint8_t* xsc, const float* xts,
+                       int64_t B, void* y, int ydt, void* ws, size_t wsb, cudaStream_t st) {
+    switch (f4_nt(B)) {
+        case 16: return run_fp4<NV, 16>(wq, wsc, wts, out, in, xq, xsc, xts, B, y, ydt, ws, wsb, st);
+        case 32: return run_fp4<NV, 32>(wq, wsc, wts, out, in, xq, xsc, xts, B, y, ydt, ws, wsb, st);
+        case 64: return run_fp4<NV, 64>(wq, wsc, wts, out, in, xq, xsc, xts, B, y, ydt, ws, wsb, st);
+        default:
+            return run_fp4<NV, 128>(wq, wsc, wts, out, in, xq, xsc, xts, B, y, ydt, ws, wsb, st);
+    }
+}
 }  // namespace
 
 extern "C" {
@@ -1185,6 +1248,48 @@ q4_status nvfp4_dequant(const uint8_t* packed, const uint8_t* scales, const floa
         return Q4_ERR_ALIGNMENT;
     return fp4_dequant<true>(packed, scales, tensor_scale, out, in, W_hat, out_dtype,
                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fp4_gemm_workspace_bytes(int32_t format, int64_t out, int64_t in, int64_t B) {
+    if ((format != Q4_FP4_MXFP4 && format != Q4_FP4_NVFP4) || out <= 0 || in <= 0 || B < 1)
+        return 0;
+    return fp4_plan(out, in, B < kF4MaxB ? B : kF4MaxB, sm_count(current_device())).ws_bytes;
+}
+
+q4_status fp4_gemm(int32_t format, const uint8_t* w_packed, const uint8_t* w_scales,
+                   const float* w_tensor_scale, int64_t out, int64_t in, const uint8_t* x_packed,
+                   const uint8_t* x_scales, const float* x_tensor_scale, int64_t B, void* y,
+                   q4_dtype y_dtype, void* workspace, size_t workspace_bytes, q4_stream stream) {
+    if (format != Q4_FP4_MXFP4 && format != Q4_FP4_NVFP4) return Q4_ERR_INVALID_ARG;
+    if (!valid_dtype(y_dtype)) return Q4_ERR_INVALID_ARG;
+    const bool nv = format == Q4_FP4_NVFP4;
+    if (out < 0 || in <= 0 || B < 1 || (in % (nv ? 256 : 512)) != 0) return Q4_ERR_SHAPE;
+    if (out == 0) return Q4_OK;
+    if (!w_packed || !w_scales || !x_packed || !x_scales || !y) return Q4_ERR_INVALID_ARG;
+    if (nv && (!w_tensor_scale || !x_tensor_scale)) return Q4_ERR_INVALID_ARG;
+    const int ysz = y_dtype == Q4_F32 ? 4 : 2;
+    if (!aligned(w_packed, 16) || !aligned(w_scales, 16) || !aligned(x_packed, 16) ||
+        !aligned(x_scales, 16) || !aligned(y, ysz) ||
+        (nv && (!aligned(w_tensor_scale, 4) || !aligned(x_tensor_scale, 4))))
+        return Q4_ERR_ALIGNMENT;
+    if (!workspace) return Q4_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int ydt = y_dtype == Q4_F32 ? 2 : (y_dtype == Q4_BF16 ? 1 : 0);
+    const int64_t vs = nv ? 16 : 32;
+    // batches beyond the MMA's N run as slices of 128 activation rows
+    for (int64_t b0 = 0; b0 < B; b0 += kF4MaxB) {
+        const int64_t nb = B - b0 < kF4MaxB ? B - b0 : kF4MaxB;
+        const uint8_t* xq = x_packed + b0 * (in / 2);
+        const uint8_t* xs = x_scales + b0 * (in / vs);
+        void* yb = reinterpret_cast<uint8_t*>(y) + b0 * out * ysz;
+        const q4_status s =
+            nv ? dispatch_fp4<true>(w_packed, w_scales, w_tensor_scale, out, in, xq, xs,
+                                    x_tensor_scale, nb, yb, ydt, workspace, workspace_bytes, st)
+               : dispatch_fp4<false>(w_packed, w_scales, nullptr, out, in, xq, xs, nullptr, nb, yb,
+                                     ydt, workspace, workspace_bytes, st);
+        if (s != Q4_OK) return s;
+    }
+    return Q4_OK;
 }
 
 q4_status q4_selftest_wait_timeout(int64_t limit_ns, q4_stream stream) {

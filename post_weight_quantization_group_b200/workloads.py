@@ -126,3 +126,25 @@ def kv_cache(batch: int, heads: int, seq: int, head_dim: int, seed: int, dtype=t
     if n_sink:
         x[:, :, :n_sink, :] *= sink_scale
     return x.to(dtype)
+
+
+# FP4 operands drawn directly as bytes, for the W4A4 product: every E2M1
+# code equally likely (both signs, -0 included) and scale bytes uniform over
+# a range -- E4M3 bytes 0x00..0x7E (zero, subnormal and normal scales up to
+# 448) for NVFP4, E8M0 bytes 112..136 (2^-15 .. 2^9) for MXFP4 -- with the
+# NVFP4 tensor scales of a weight (max |W| ~ 0.1) and of an activation
+# (max |x| ~ 20) matrix.
+FP4_BLOCK = {"mxfp4": 32, "nvfp4": 16}
+FP4_SCALE_BYTES = {"mxfp4": (112, 136), "nvfp4": (0x00, 0x7E)}
+FP4_W_TENSOR_SCALE = 0.1 / 2688.0
+FP4_X_TENSOR_SCALE = 20.0 / 2688.0
+
+
+def fp4_operand(rows: int, inn: int, fmt: str, seed: int):
+    """(packed codes uint8 [rows, in/2], scale bytes uint8 [rows, in/block]) on the CPU."""
+    g = _gen(seed, "cpu")
+    packed = torch.randint(0, 256, (rows, inn // 2), generator=g, dtype=torch.uint8)
+    lo, hi = FP4_SCALE_BYTES[fmt]
+    scales = torch.randint(lo, hi + 1, (rows, inn // FP4_BLOCK[fmt]), generator=g,
+                           dtype=torch.uint8)
+    return packed, scales
