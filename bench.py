@@ -11,6 +11,17 @@ the fp16 copies freed; activations are bf16 N(0, 1).
                     [--workload llama3-8b | llama3-70b-stack [--batch B]]
                     [--layers L] [--no-sweep] [--no-cpu-baseline]
 
+Single operations for profiling: --workload q4-70b-down [--batch B]
+[--group-size G] [--asym], w8a16-70b, nvfp4-70b-down, mxfp4-70b-down,
+kv8-70b-32k.
+
+A step launches, per layer, q/k/v as one q4_gemv_grouped call, o, gate/up as
+one grouped call and down (4 launches; the 7-launch form is reported beside
+it as ``ungrouped``).  The default run also reports the INT4/bf16 batch
+sweep, act order, the fused layout, W8A16, the KV-cache and FP4 quantizers,
+the W4A4 FP4 product against batch, and the Llama-3-70B decode stack (80
+layers, asymmetric group 64) at B = 1 and 8.
+
 Prints one JSON line (rank 0).  ``value`` is the aggregate HBM throughput of
 the INT4 products (algorithmic bytes / device time, CUDA events, max over
 ranks); ``us_per_layer`` the time of one decoder layer's seven products.
@@ -37,15 +48,15 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# DRAM traffic of q4_gemv_sk_kernel per algorithmic byte, from the ncu capture
-# of a launch of this workload (dram__bytes_read.sum + dram__bytes_write.sum =
-# 30.33 MB on a 14336 x 4096 gate_proj launch whose algorithmic bytes are
-# 30.28 MB).  Shapes with few row tiles write stream-K partials too (the
-# 70B down_proj capture: reads 1.018x, plus 3.8 MB of partials).  Scaled to
-# the bench's average launch; it must be re-taken whenever the kernel changes.
-GEMV_TRAFFIC_RATIO = 30.33 / 30.28
-GEMV_TRAFFIC_SOURCE = ("ncu --set full on one 14336x4096 B=1 launch "
-                       "(profiles/q4_gemv_sk_llama3_8b_gate_full.txt)")
+# DRAM traffic of q4_gemv_sk_kernel per algorithmic byte, from the ncu
+# capture of the four launches of one Llama-3-8B layer as the step launches
+# them (q/k/v grouped, o, gate/up grouped, down): dram__bytes_read.sum +
+# dram__bytes_write.sum = 113.11 MB against 112.62 MB of algorithmic bytes.
+# Scaled to the step's average launch; it must be re-taken whenever the
+# kernel changes.
+GEMV_TRAFFIC_RATIO = 113.10976 / 112.623616
+GEMV_TRAFFIC_SOURCE = ("ncu --set full on the 4 launches of one B=1 layer "
+                       "(profiles/q4_gemv_sk_llama3_8b_layer_grouped_full.txt)")
 
 
 def load_peaks():
@@ -154,6 +165,28 @@ def build_llama3_8b(q4, wl, torch, layers, rank, B, device):
           for name, (out, _) in wl.LLAMA3_8B.items()}
     torch.cuda.synchronize()
     return mats, xs, ys
+
+
+def layer_plan(mats, xs, ys):
+    """Launch plan of a decode step over `mats` (7 linears per layer in
+    q,k,v,o,gate,up,down order): q/k/v in one grouped call, o, gate/up in one
+    grouped call, down -- 4 launches per layer."""
+    plan = []
+    for l in range(0, len(mats), 7):
+        m = dict(mats[l:l + 7])
+        for names in (("q_proj", "k_proj", "v_proj"), ("o_proj",), ("gate_proj", "up_proj"),
+                      ("down_proj",)):
+            ws_ = [m[n] for n in names]
+            plan.append((ws_, [ys[n] for n in names], xs[ws_[0].in_features]))
+    return plan
+
+
+def run_plan(q4, plan, wsp):
+    for ws_, ys_, x in plan:
+        if len(ws_) > 1:
+            q4.q4_gemv_grouped(ws_, x, ys=ys_, workspace=wsp)
+        else:
+            q4.q4_gemm_skinny(ws_[0], x, y=ys_[0], workspace=wsp)
 
 
 def time_region(torch, fn, steps, warmup, stream):
@@ -411,6 +444,110 @@ def fp4_cost(q4, wl, torch, device, stream, hbm_peak):
                                      "nvfp4_dequant": round(b_nvd / t_nvd / 1e3 / hbm_peak, 4)}}
 
 
+FP4_SWEEP_B = (1, 16, 32, 64, 128)
+
+
+def fp4_w4a4_sweep(q4, wl, torch, device, stream, hbm_peak):
+    """W4A4 product (fp4_gemm, block-scaled tcgen05 MMA) against batch on the
+    Llama-3-70B down_proj and gate_proj shapes, NVFP4 and MXFP4: seeded FP4
+    weight bytes (every code, the formats' scale-byte ranges), activations
+    N(0, 1) bf16 quantized by the library (timed separately: the activation
+    quantization a W4A4 decode step adds), four weight copies rotating so no
+    call finds its weights in L2.  Algorithmic bytes: codes and scale bytes
+    of W and x, bf16 y."""
+    res = {}
+    for name in ("down_proj", "gate_proj"):
+        out, inn = wl.LLAMA3_70B[name]
+        for fmt in ("nvfp4", "mxfp4"):
+            ws = []
+            for i in range(4):
+                p_, s_ = wl.fp4_operand(out, inn, fmt, 40 + i)
+                ts = (torch.tensor([wl.FP4_W_TENSOR_SCALE], dtype=torch.float32, device=device)
+                      if fmt == "nvfp4" else None)
+                ws.append(q4.FP4Weight(p_.to(device), s_.to(device), out, inn, fmt, ts))
+            rows = {}
+            for B in FP4_SWEEP_B:
+                xb = wl.activations(B, inn, 31, device=device)
+                X = q4.fp4_quantize(xb, fmt)
+                y = torch.empty(B, out, dtype=torch.bfloat16, device=device)
+                wsp = q4.fp4_workspace_for(ws[0], B, device)
+                t = graph_time_us(torch, lambda i: q4.fp4_gemm(ws[i % 4], X, y=y, workspace=wsp),
+                                  16, stream)
+                tq = graph_time_us(torch, lambda i: q4.fp4_quantize(xb, fmt), 16, stream)
+                nb = fp4_bytes(out, inn, fmt, B)
+                rows[B] = {"us": round(t, 2), "gbs": round(nb / t / 1e3, 1),
+                           "frac_of_measured_hbm": round(nb / t / 1e3 / hbm_peak, 4),
+                           "tflops": round(2 * B * out * inn / t / 1e6, 1),
+                           "x_quantize_us": round(tq, 2)}
+            res[f"{name}.{fmt}"] = {"shape": f"{out}x{inn}", "by_B": rows}
+            del ws
+    st = q4.q4_sync_status()
+    assert st == q4.Q4_OK, q4.status_string(st)
+    return res
+
+
+def build_llama3_70b_stack(q4, wl, torch, device):
+    """80 distinct Llama-3-70B layers x 7 linears, asymmetric group 64: N(0,
+    0.02^2) fp16 weights generated on the device per linear (seed 1000 layer
+    + linear index), quantized, fp16 freed (34.2 GB of codes, scales, zeros)."""
+    mats = []
+    for layer in range(wl.LLAMA3_70B_LAYERS):
+        for idx, (name, (out, inn)) in enumerate(wl.LLAMA3_70B.items()):
+            W = wl.normal_weight(out, inn, wl.llama3_70b_stack_seed(layer, idx), device=device)
+            mats.append((name, q4.q4_quantize_pack(W, 64, False)))
+            del W
+    torch.cuda.synchronize()
+    return mats
+
+
+def stack_cost(q4, wl, torch, device, stream, B, steps, hbm_peak, mats=None):
+    """One Llama-3-70B decode step over the 80-layer stack at batch B, as one
+    CUDA graph: grouped launches (q/k/v and gate/up in one call each, 320
+    launches) and, beside it, one launch per linear (560)."""
+    own = mats is None
+    if own:
+        mats = build_llama3_70b_stack(q4, wl, torch, device)
+    shapes = wl.LLAMA3_70B
+    xs = {inn: wl.activations(B, inn, 17 + inn, device=device) for _, (_, inn) in shapes.items()}
+    ys = {name: torch.empty(B, out, dtype=torch.bfloat16, device=device)
+          for name, (out, _) in shapes.items()}
+    wsp = q4.workspace_for(mats[0][1], B, device)
+    step_bytes = sum(algo_bytes(*shapes[n], 64, B, sym=False) for n, _ in mats)
+    plan = layer_plan(mats, xs, ys)
+
+    def grouped():
+        run_plan(q4, plan, wsp)
+
+    def single():
+        for name, w in mats:
+            q4.q4_gemm_skinny(w, xs[shapes[name][1]], y=ys[name], workspace=wsp)
+
+    res = {"batch": B, "bytes_per_step": step_bytes, "group_size": 64, "symmetric": False}
+    for key, fn, nl in (("grouped", grouped, len(plan)), ("per_linear", single, len(mats))):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        st = q4.q4_sync_status()
+        assert st == q4.Q4_OK, q4.status_string(st)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            fn()
+        torch.cuda.synchronize()
+        with ClockSampler(device.index or 0) as clk:
+            ms = time_region(torch, g.replay, steps, 3, stream) / steps
+        del g
+        gbs = step_bytes / (ms * 1e-3) / 1e9
+        res[key] = {"ms_per_step": round(ms, 4), "us_per_layer": round(ms * 1e3 / 80, 2),
+                    "gbs": round(gbs, 1), "frac_of_measured_hbm": round(gbs / hbm_peak, 4),
+                    "launches_per_step": nl, "steps": steps, "clocks": clk.summary()}
+    st = q4.q4_sync_status()
+    assert st == q4.Q4_OK, q4.status_string(st)
+    if own:
+        del mats
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -437,11 +574,16 @@ def run_ours(args):
     mats, xs, ys = build_llama3_8b(q4, wl, torch, layers, rank, B, device)
     shapes = wl.LLAMA3_8B
     step_bytes = sum(algo_bytes(*shapes[n], 128, B) for n, _ in mats)
-    launches_per_step = len(mats)
+    wsp = q4.workspace_for(mats[0][1], B, device)
+    plan = layer_plan(mats, xs, ys)
+    launches_per_step = len(plan)
 
     def step():
+        run_plan(q4, plan, wsp)
+
+    def step_ungrouped():
         for name, w in mats:
-            q4.q4_gemv(w, xs[shapes[name][1]], y=ys[name])
+            q4.q4_gemv(w, xs[shapes[name][1]], y=ys[name], workspace=wsp)
 
     # eager warm-up (loads modules, sets kernel attributes), then capture
     for _ in range(3):
@@ -464,6 +606,16 @@ def run_ours(args):
     assert st == q4.Q4_OK, q4.status_string(st)
     ms_eager = time_region(torch, step, max(3, args.steps // 10), 2, stream)
     ms_eager /= max(3, args.steps // 10)
+    # the same products launched one per linear (7 per layer)
+    for _ in range(3):
+        step_ungrouped()
+    torch.cuda.synchronize()
+    ugraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ugraph, capture_error_mode="thread_local"):
+        step_ungrouped()
+    nu = max(20, args.steps // 4)
+    ms_ungrouped = time_region(torch, ugraph.replay, nu, 3, stream) / nu
+    del ugraph
 
     ms_max = max_over_ranks(ms, dist, device)
     ms_per_step = ms_max / args.steps
@@ -562,7 +714,9 @@ def run_ours(args):
         "data": "synthetic (seeded N(0,0.02^2) fp16 weights quantized on device; bf16 N(0,1) activations)",
         "config": {"workload": f"Llama-3-8B decode linears q,k,v,o,gate,up,down x {layers} distinct layers per step",
                    "batch": B, "group_size": 128, "symmetric": True, "layers": layers,
-                   "linears_per_step": launches_per_step,
+                   "linears_per_step": len(mats), "launches_per_step": launches_per_step,
+                   "launch_plan": "per layer: q4_gemv_grouped(q,k,v), q4_gemv(o), "
+                                  "q4_gemv_grouped(gate,up), q4_gemv(down)",
                    "bytes_per_step": step_bytes, "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB of packed weights per step, 126 MB L2)",
                    "timing": "CUDA graph of the step, CUDA events on the launching stream"},
@@ -570,6 +724,9 @@ def run_ours(args):
         "pct_of_8TBs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
         "pct_of_measured_hbm": round(100 * value / world / peak, 2),
         "eager_us_per_layer": round(ms_eager / layers * 1e3, 3),
+        "ungrouped": {"us_per_layer": round(ms_ungrouped / layers * 1e3, 3),
+                      "gbs": round(step_bytes / (ms_ungrouped * 1e-3) / 1e9, 1),
+                      "launches_per_step": len(mats)},
         "bf16": {"us_per_layer": round(min(ms_bf, ms_cublas) * 1e3, 3),
                  "gbs": round(bf_bytes / (min(ms_bf, ms_cublas) * 1e-3) / 1e9, 1),
                  "speedup_int4_vs_bf16_B1": round(min(ms_bf, ms_cublas) / int4_layer_ms, 3),
@@ -584,13 +741,9 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": round(value / world, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(value / world / peak, 4),
                      "peak_kind": peak_kind,
-                     # the kernel changed (nibble shifts moved to the ALU) after its last
-                     # ncu capture: no current counters, so no traffic figure
-                     "traffic": None,
+                     "traffic": round(GEMV_TRAFFIC_RATIO * step_bytes / launches_per_step),
                      "traffic_unit": "DRAM bytes per launch",
-                     "traffic_note": ("kernel changed since the last ncu capture; that capture "
-                                      "(previous version, same memory accesses) measured "
-                                      f"{GEMV_TRAFFIC_RATIO:.3f} x the algorithmic bytes: "
+                     "traffic_note": (f"{GEMV_TRAFFIC_RATIO:.4f} x the algorithmic bytes: "
                                       + GEMV_TRAFFIC_SOURCE),
                      "kernel": "q4_gemv_sk_kernel<bf16,g128,sym,8,1>",
                      "bytes_per_launch_avg": step_bytes // launches_per_step},
@@ -608,6 +761,13 @@ def run_ours(args):
             out["w8a16"] = w8a16_cost(q4, wl, torch, device, stream, peak)
             out["kv_cache"] = kv_cache_cost(q4, wl, torch, device, stream, peak)
             out["fp4"] = fp4_cost(q4, wl, torch, device, stream, peak)
+            out["fp4_w4a4_by_B"] = fp4_w4a4_sweep(q4, wl, torch, device, stream, peak)
+            stack = build_llama3_70b_stack(q4, wl, torch, device)
+            out["llama3_70b_stack"] = {
+                f"B{b}": stack_cost(q4, wl, torch, device, stream, b, max(10, args.steps // 100),
+                                    peak, mats=stack) for b in (1, 8)}
+            del stack
+            torch.cuda.empty_cache()
         out["cpu_baseline"] = cpu_baseline() if (world == 1 and not args.no_cpu_baseline) else None
         print(json.dumps(out), flush=True)
     del graph
@@ -634,13 +794,7 @@ def run_stack(args):
     stream = torch.cuda.current_stream()
     B, g = args.batch, 64
     shapes = wl.LLAMA3_70B
-    mats = []
-    for layer in range(80):
-        for idx, (name, (out, inn)) in enumerate(shapes.items()):
-            W = wl.normal_weight(out, inn, wl.llama3_70b_stack_seed(layer, idx), device=device)
-            mats.append((name, q4.q4_quantize_pack(W, g, False)))
-            del W
-    torch.cuda.synchronize()
+    mats = build_llama3_70b_stack(q4, wl, torch, device)
     xs = {inn: wl.activations(B, inn, 17 + inn, device=device) for _, (_, inn) in shapes.items()}
     ys = {name: torch.empty(B, out, dtype=torch.bfloat16, device=device) for name, (out, _) in shapes.items()}
     ws = q4.workspace_for(mats[0][1], B, device)
@@ -738,6 +892,60 @@ def _oracle_pass(prepared, frac=1.0):
     return nbytes
 
 
+def host_cpu():
+    """nproc and the lscpu model name of the host the oracle runs on."""
+    model = None
+    try:
+        txt = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for ln in txt.splitlines():
+            if ln.startswith("Model name:"):
+                model = ln.split(":", 1)[1].strip()
+    except (OSError, subprocess.SubprocessError):
+        pass
+    return {"nproc": os.cpu_count(), "lscpu_model": model, "threads_used": 1}
+
+
+def _oracle_small_case():
+    """The 512 x 1024 parity case (N(0, 0.02^2) fp16, sym g128, B=1, CPU
+    generator seed 0), quantized and multiplied whole by the oracle: seconds."""
+    import numpy as np
+    import torch
+    import oracle
+    from post_weight_quantization_group_b200 import workloads as wl
+    W = wl.normal_weight(512, 1024, 0).float().numpy()
+    x = wl.activations(1, 1024, 0, dtype=torch.float16).float().numpy().astype(np.float64)
+    t0 = time.perf_counter()
+    q, s_, _ = oracle.quantize_pack(W, 128, True)
+    oracle.gemv(q, s_, None, 512, 1024, 128, True, x)
+    return time.perf_counter() - t0
+
+
+def _oracle_stack_sample(frac=1.0 / 16):
+    """Layer 0 of the Llama-3-70B stack (asym g64, B=1): the first `frac` of
+    every linear's rows (weights from the stack's seeds), quantized by the
+    oracle (not timed), then its fp64 product (timed).  Returns (seconds,
+    algorithmic bytes of the sample)."""
+    import numpy as np
+    import torch
+    import oracle
+    from post_weight_quantization_group_b200 import workloads as wl
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    prepared = []
+    for idx, (name, (out, inn)) in enumerate(wl.LLAMA3_70B.items()):
+        n = max(1, int(out * frac))
+        W = wl.normal_weight(out, inn, wl.llama3_70b_stack_seed(0, idx), device=dev)[:n]
+        q, s_, z = oracle.quantize_pack(W.float().cpu().numpy(), 64, False)
+        x = wl.activations(1, inn, 17 + inn).float().numpy().astype(np.float64)
+        prepared.append((n, inn, q, s_, z, x))
+        del W
+    t0 = time.perf_counter()
+    nbytes = 0
+    for n, inn, q, s_, z, x in prepared:
+        oracle.gemv(q, s_, z, n, inn, 64, False, x)
+        nbytes += algo_bytes(n, inn, 64, 1, sym=False)
+    return time.perf_counter() - t0, nbytes
+
+
 def cpu_baseline():
     prepared = _oracle_layer()
     t0 = time.perf_counter()
@@ -745,10 +953,24 @@ def cpu_baseline():
     for _ in range(3):
         nbytes += _oracle_pass(prepared)
     dt = time.perf_counter() - t0
+    frac = 1.0 / 16
+    t5, b5 = _oracle_stack_sample(frac)
     return {"value": round(nbytes / dt / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": "3 passes over 1 of 32 Llama-3-8B layers (7 linears, sym g128, B=1), "
                       "fp64 product of the CPU oracle, single thread",
-            "seconds": round(dt, 2)}
+            "seconds": round(dt, 2), "host": host_cpu(),
+            "small_case_512x1024_seconds": round(_oracle_small_case(), 4),
+            "llama3_70b_stack_B1": {
+                "sample": "first 1/16 of the rows of each of the 7 linears of layer 0 "
+                          "(asym g64, B=1), fp64 product, single thread",
+                "seconds": round(t5, 2), "gbs": round(b5 / t5 / 1e9, 4),
+                "seconds_per_step_extrapolated": round(t5 / frac * wl_layers_70b(), 1),
+                "extrapolation": "x16 (rows) x 80 (layers)"}}
+
+
+def wl_layers_70b():
+    from post_weight_quantization_group_b200 import workloads as wl
+    return wl.LLAMA3_70B_LAYERS
 
 
 def run_reference(args):
@@ -793,8 +1015,8 @@ def run_op(args):
     """One operation of the path alone, for profiling and spot timing:
     ``w8a16-70b`` = q8_gemv on the Llama-3-70B down_proj (8192 x 28672, batch
     --batch, two weight copies rotating); ``q4-70b-down`` = q4_gemm_skinny
-    (sym g128) on the same shape and batch (the B <= 8 kernel or, above, the
-    tcgen05 kernel); ``nvfp4-70b-down`` / ``mxfp4-70b-down`` = fp4_gemm (W4A4,
+    (--group-size, symmetric unless --asym) on the same shape and batch (the
+    B <= 8 kernel or, above, the tcgen05 kernel); ``nvfp4-70b-down`` / ``mxfp4-70b-down`` = fp4_gemm (W4A4,
     seeded FP4 weight bytes, activations quantized by the library) on the same
     shape and batch; ``kv8-70b-32k`` = kv_quantize_int8
     of one layer's K cache at 32768 tokens ([1, 8, 32768, 128] bf16, four
@@ -824,8 +1046,8 @@ def run_op(args):
         name, cfg = "W8A16 per-channel INT8 GEMV", {"workload": f"Llama-3-70B down_proj {out}x{inn}", "batch": B}
     elif args.workload == "q4-70b-down":
         out, inn = wl.LLAMA3_70B["down_proj"]
-        B = args.batch
-        ws = [q4.q4_quantize_pack(wl.normal_weight(out, inn, 30 + i, device=device), 128, True)
+        B, g, sym = args.batch, args.group_size, not args.asym
+        ws = [q4.q4_quantize_pack(wl.normal_weight(out, inn, 30 + i, device=device), g, sym)
               for i in range(2)]
         torch.cuda.empty_cache()
         x = wl.activations(B, inn, 31, device=device)
@@ -833,8 +1055,10 @@ def run_op(args):
         wsp = q4.workspace_for(ws[0], B, device)
         it = iter(range(1 << 30))
         fn = lambda: q4.q4_gemm_skinny(ws[next(it) % 2], x, y=y, workspace=wsp)
-        nbytes = algo_bytes(out, inn, 128, B)
-        name, cfg = "W4A16 INT4 product (sym g128)", {"workload": f"Llama-3-70B down_proj {out}x{inn}", "batch": B}
+        nbytes = algo_bytes(out, inn, g, B, sym=sym)
+        kind = f"{'sym' if sym else 'asym'} g{g}"
+        name, cfg = (f"W4A16 INT4 product ({kind})",
+                     {"workload": f"Llama-3-70B down_proj {out}x{inn}", "batch": B, "quant": kind})
     elif args.workload in ("nvfp4-70b-down", "mxfp4-70b-down"):
         fmt = args.workload.split("-")[0]
         out, inn = wl.LLAMA3_70B["down_proj"]
@@ -884,7 +1108,12 @@ def main():
     ap.add_argument("--workload", default="llama3-8b",
                     choices=["llama3-8b", "llama3-70b-stack", "w8a16-70b", "q4-70b-down",
                              "kv8-70b-32k", "nvfp4-70b-down", "mxfp4-70b-down"])
-    ap.add_argument("--batch", type=int, default=1, help="batch of the llama3-70b-stack workload")
+    ap.add_argument("--batch", type=int, default=1,
+                    help="batch of the llama3-70b-stack and single-op workloads")
+    ap.add_argument("--group-size", type=int, default=128, choices=[32, 64, 128],
+                    help="INT4 group size of the q4-70b-down workload")
+    ap.add_argument("--asym", action="store_true",
+                    help="asymmetric (zero-point) INT4 in the q4-70b-down workload")
     ap.add_argument("--layers", type=int, default=32,
                     help="distinct decoder layers per step (32 = the Llama-3-8B depth)")
     ap.add_argument("--no-sweep", action="store_true",

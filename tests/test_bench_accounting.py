@@ -55,3 +55,28 @@ def test_peaks_fall_back_without_measurements(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     peaks, kind = bench.load_peaks()
     assert kind == "fallback" and peaks["hbm_gbs"] == 6650.0
+
+
+def test_fp4_bytes():
+    # codes (out + B) in/2, scale bytes (out + B) in/block, y bf16
+    assert bench.fp4_bytes(8192, 28672, "nvfp4", 16) == (8192 + 16) * (14336 + 1792) + 16 * 8192 * 2
+    assert bench.fp4_bytes(8192, 28672, "mxfp4", 1) == 8193 * (14336 + 896) + 8192 * 2
+
+
+def test_layer_plan_groups_qkv_and_gate_up():
+    class W:
+        def __init__(self, name, inn):
+            self.name, self.in_features = name, inn
+
+    mats = [(n, W(n, i)) for _ in range(2) for n, (o, i) in wl.LLAMA3_8B.items()]
+    xs = {4096: "x4096", 14336: "x14336"}
+    ys = {n: "y_" + n for n in wl.LLAMA3_8B}
+    plan = bench.layer_plan(mats, xs, ys)
+    assert len(plan) == 8
+    assert [[w.name for w in p[0]] for p in plan[:4]] == [
+        ["q_proj", "k_proj", "v_proj"], ["o_proj"], ["gate_proj", "up_proj"], ["down_proj"]]
+    assert [p[1] for p in plan[:4]] == [["y_q_proj", "y_k_proj", "y_v_proj"], ["y_o_proj"],
+                                        ["y_gate_proj", "y_up_proj"], ["y_down_proj"]]
+    assert plan[0][2] == "x4096" and plan[3][2] == "x14336"
+    # the second layer's products, not the first one's again
+    assert plan[4][0][0] is mats[7][1] and plan[7][0][0] is mats[13][1]

@@ -211,12 +211,15 @@ def test_gemv_llama3_70b_heavy_tail(name, g, B):
                rows=_sample_rows(out, 128), n_outliers=4)
 
 
+@pytest.mark.parametrize("layer", [0, 39, 79])
 @pytest.mark.parametrize("idx,name", list(enumerate(wl.LLAMA3_70B)))
 @pytest.mark.parametrize("B", [1, 8])
-def test_gemv_llama3_70b_stack_asym_g64(idx, name, B):
+def test_gemv_llama3_70b_stack_asym_g64(layer, idx, name, B):
+    """The Llama-3-70B decode stack's weights (asymmetric group 64) of the
+    first, middle and last layer, generated from the stack's seeds."""
     out, inn = wl.LLAMA3_70B[name]
-    _gemv_case(out, inn, 64, False, B, torch.bfloat16, seed=wl.llama3_70b_stack_seed(0, idx),
-               rows=_sample_rows(out, 96))
+    _gemv_case(out, inn, 64, False, B, torch.bfloat16, seed=wl.llama3_70b_stack_seed(layer, idx),
+               rows=_sample_rows(out, 96, seed=layer))
 
 
 def test_gemv_special_inputs():
