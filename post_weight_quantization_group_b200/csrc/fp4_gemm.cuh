@@ -138,6 +138,12 @@ __device__ __forceinline__ void bulk_load_g2s(uint32_t dst, const void* src, uin
         : "memory");
 }
 
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // Orders this thread's earlier generic-proxy memory accesses before its
 // later async-proxy ones (bulk copies).
 __device__ __forceinline__ void fence_proxy_async() {
@@ -442,7 +448,28 @@ __global__ void __launch_bounds__(kF4Threads, 1)
             const int64_t row = static_cast<int64_t>(tile) * kF4RT + r;
             const int slot = static_cast<int>(2 * p + (first ? 0 : 1));
             float* part = ws_part + static_cast<size_t>(slot) * kF4RT * NT;
-            if (ok) {
+            const int64_t t64 = tile;
+            const int64_t q_lo = sk_owner(t64 * nchunks, T, P);
+            const int64_t q_hi = sk_owner(t64 * nchunks + nchunks - 1, T, P);
+            const int nothers = static_cast<int>(q_hi - q_lo);
+            // at the end of the range every stage has been consumed: the
+            // other partials are bulk-copied into shared memory at once
+            const bool bulk = final_seg && nothers <= fix_cap;
+            // A final partial segment whose tile counter already holds every
+            // other contributor is certainly the last one: it keeps its
+            // partial in tensor memory instead of storing it.
+            bool early = false;
+            if (!whole && bulk) {
+                named_bar_sync(1, 128);
+                if (threadIdx.x == 192) {
+                    const bool e = ld_acquire_gpu(ws_count + tile) == static_cast<unsigned>(nothers);
+                    if (e) ws_count[tile] = 0u;  // no other contributor touches it again
+                    *last_flag = e ? 2u : 0u;
+                }
+                named_bar_sync(1, 128);
+                early = *last_flag == 2u;
+            }
+            if (ok && !(early && !whole)) {
 #pragma unroll 1
                 for (int c0 = 0; c0 < NT; c0 += PW) {
                     uint32_t v[PW];
@@ -471,19 +498,15 @@ __global__ void __launch_bounds__(kF4Threads, 1)
                 if (lane == 0) mbar_arrive(&acc_empty[a]);
             }
             if (!whole) {
-                const int64_t t64 = tile;
-                const int64_t q_lo = sk_owner(t64 * nchunks, T, P);
-                const int64_t q_hi = sk_owner(t64 * nchunks + nchunks - 1, T, P);
-                const int nothers = static_cast<int>(q_hi - q_lo);
-                // at the end of the range every stage has been consumed: the
-                // other partials are bulk-copied into shared memory at once
-                const bool bulk = final_seg && nothers <= fix_cap;
                 named_bar_sync(1, 128);
                 if (threadIdx.x == 192) {
-                    const unsigned prev = atom_add_acq_rel_gpu(ws_count + tile, 1u);
-                    const bool last = prev == static_cast<unsigned>(nothers);
+                    bool last = early;
+                    if (!early) {
+                        const unsigned prev = atom_add_acq_rel_gpu(ws_count + tile, 1u);
+                        last = prev == static_cast<unsigned>(nothers);
+                        if (last) ws_count[tile] = 0u;  // zero again for the next call
+                    }
                     *last_flag = last ? 1u : 0u;
-                    if (last) ws_count[tile] = 0u;  // zero again for the next call
                     if (last && bulk) {
                         fence_proxy_async();  // the partials were written through the generic proxy
                         mbar_arrive_expect_tx(fixbar,
