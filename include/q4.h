@@ -307,14 +307,21 @@ Q4_API q4_status q4_gemv_noalloc(const q4_weight* w, const void* x, q4_dtype x_d
  * The unquantised bf16 product y = x W^T with fp32 accumulation, a
  * baseline the INT4 path is compared against and the probe of the bandwidth
  * a weight stream reaches (ybb.press section 一, roofline_bound; arganzheng.
- * life section 二.4, BF16 vs W4A16 batch table).
+ * life section 二.4, BF16 vs W4A16 batch table).  W and x tiles go by TMA to
+ * shared memory and straight into the tcgen05 tensor cores (fp32 accumulator
+ * in tensor memory), split over a persistent grid like the INT4 products.
  *   W [out, in] bf16, x [B, in] bf16, y [B, out] bf16; `in` a multiple of 64;
- *   W, x, y 16-byte aligned.
- *   1 <= B <= 8 runs here; 9 <= B <= 128 returns Q4_ERR_UNSUPPORTED (a plain
- *   library GEMM is the bf16 baseline there); other B Q4_ERR_SHAPE.
+ *   W, x, y 16-byte aligned; 1 <= B <= 128 (else Q4_ERR_SHAPE).
+ *   workspace  at least bf16_ref_workspace_bytes(out, in, B) bytes, 256-byte
+ *              aligned, zero-filled before its first use (the kernel leaves
+ *              its counters zero again); the same layout as the INT4
+ *              products' workspace, so one buffer serves both.
+ * Deterministic: split tiles add their partials in a fixed order.
  */
+Q4_API size_t bf16_ref_workspace_bytes(int64_t out, int64_t in, int64_t B);
 Q4_API q4_status bf16_gemv_ref_bw(const void* W, int64_t out, int64_t in, const void* x, int64_t B,
-                           void* y, q4_stream stream);
+                                  void* y, void* workspace, size_t workspace_bytes,
+                                  q4_stream stream);
 
 /* ------------------------------------------------ per-channel INT8 weights
  *

@@ -43,7 +43,7 @@ ABI_SYMBOLS = (
     "q4_permute_activations", "q8_quantize_per_channel", "q8_dequant", "q8_workspace_bytes",
     "q8_gemv", "kv_quantize_int8", "kv_dequant_int8", "kv_quantize_int4", "kv_dequant_int4",
     "mxfp4_quantize", "mxfp4_dequant", "nvfp4_quantize", "nvfp4_dequant", "q4_gemv_grouped",
-    "fp4_gemm_workspace_bytes", "fp4_gemm",
+    "fp4_gemm_workspace_bytes", "fp4_gemm", "bf16_ref_workspace_bytes",
 )
 
 
@@ -98,7 +98,9 @@ def load_library(path: str = LIB_PATH):
     lib.q4_gemv_grouped.argtypes = [W, I32, P, S, I64, ctypes.POINTER(P), S, P, ctypes.c_size_t, P]
     lib.q4_workspace_bytes.argtypes = [I64, I64, I64, I32]
     lib.q4_workspace_bytes.restype = ctypes.c_size_t
-    lib.bf16_gemv_ref_bw.argtypes = [P, I64, I64, P, I64, P, P]
+    lib.bf16_gemv_ref_bw.argtypes = [P, I64, I64, P, I64, P, P, ctypes.c_size_t, P]
+    lib.bf16_ref_workspace_bytes.argtypes = [I64, I64, I64]
+    lib.bf16_ref_workspace_bytes.restype = ctypes.c_size_t
     lib.q4_sync_status.argtypes = [P]
     lib.q4_selftest_wait_timeout.argtypes = [I64, P]
     lib.q8_quantize_per_channel.argtypes = [P, S, I64, I64, P, P, P]
@@ -390,15 +392,18 @@ def q4_gemv_noalloc(w: Q4Weight, x: torch.Tensor, y: torch.Tensor | None = None,
 
 
 def bf16_gemv_ref_bw(W: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None,
-                     stream=None) -> torch.Tensor:
-    """y = x W^T for bf16 W [out, in], x [B, in], B <= 8 (larger B:
-    Q4_ERR_UNSUPPORTED)."""
+                     workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = x W^T for bf16 W [out, in], x [B, in], 1 <= B <= 128, on the
+    tcgen05 tensor cores (the C entry point bf16_gemv_ref_bw)."""
     lib = load_library()
     out, inn = W.shape
     B = x.shape[0]
     if y is None:
         y = torch.empty(B, out, dtype=torch.bfloat16, device=x.device)
-    st = lib.bf16_gemv_ref_bw(_ptr(W), out, inn, _ptr(x), B, _ptr(y), _stream(stream))
+    if workspace is None:
+        workspace = _shared_workspace(int(lib.bf16_ref_workspace_bytes(out, inn, B)), x.device)
+    st = lib.bf16_gemv_ref_bw(_ptr(W), out, inn, _ptr(x), B, _ptr(y), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "bf16_gemv_ref_bw")
     return y
 

@@ -1,7 +1,7 @@
 // q4_api.cu -- the C ABI of include/q4.h: argument validation, launch
 // planning, TMA descriptor encoding and kernel launches.  All kernels live in
 // this translation unit (q4_quant.cuh, q4_gemv.cuh, q4_gemv_sk.cuh,
-// q4_skinny_tc.cuh, q8_gemv.cuh, q8_quant.cuh, fp4_quant.cuh, fp4_gemm.cuh).
+// q4_skinny_tc.cuh, q8_gemv.cuh, q8_quant.cuh, fp4_quant.cuh, tc_gemm.cuh).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -21,7 +21,7 @@
 #include "q8_gemv.cuh"
 #include "q8_quant.cuh"
 #include "fp4_quant.cuh"
-#include "fp4_gemm.cuh"
+#include "tc_gemm.cuh"
 
 namespace {
 
@@ -122,21 +122,6 @@ bool set_kernel_attrs(K kernel, int smem_bytes, bool nonportable_cluster) {
     return true;
 }
 
-// Split-K plan for the streaming kernels: rows per CTA `rt`, `nchunks` chunks
-// of K.  S CTAs of one cluster share a row tile; aim for >= 2 CTAs per SM.
-struct SplitPlan {
-    int S, cps;
-};
-
-SplitPlan plan_split(int64_t out, int nchunks, int rt, int sms) {
-    const int64_t row_tiles = (out + rt - 1) / rt;
-    int S = 1;
-    while (S < 8 && row_tiles * S < 2LL * sms && nchunks >= 2 * S) S *= 2;
-    int cps = (nchunks + S - 1) / S;
-    S = (nchunks + cps - 1) / cps;
-    return {S, cps};
-}
-
 // Launch with an optional cluster shape and, for kernels written for it,
 // programmatic stream serialization (the kernel may start before the previous
 // kernel of the stream has finished; it waits with griddepcontrol.wait).
@@ -165,13 +150,6 @@ q4_status launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem
     cfg.attrs = n ? attr : nullptr;
     cfg.numAttrs = n;
     return launch_status(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
-}
-
-template <typename... KArgs, typename... Args>
-q4_status launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                         int cluster_x, cudaStream_t stream, Args&&... args) {
-    return launch_ex(kernel, grid, block, smem, cluster_x, false, stream,
-                     std::forward<Args>(args)...);
 }
 
 bool valid_dtype(int d) { return d == Q4_F16 || d == Q4_BF16 || d == Q4_F32; }
@@ -261,20 +239,6 @@ q4_status run_quantize_clip(const void* W, int64_t out, int64_t in, int g, int n
 
 // ------------------------------------------------------------------ GEMV
 // Tile shape of the small-batch kernels (compile-time tunables).
-#ifndef Q4_GEMV_MT
-#define Q4_GEMV_MT 2
-#endif
-#ifndef Q4_GEMV_CW
-#define Q4_GEMV_CW 4
-#endif
-#ifndef Q4_GEMV_STAGES
-#define Q4_GEMV_STAGES 4
-#endif
-constexpr int kGemvMT = Q4_GEMV_MT;
-constexpr int kGemvCW = Q4_GEMV_CW;
-constexpr int kGemvStages = Q4_GEMV_STAGES;
-constexpr int kGemvRT = kGemvCW * kGemvMT * 16;
-
 // Small-batch stream-K kernel: CW consumer warps (16 rows each), 2 CTAs/SM.
 #ifndef Q4_SK_CW
 #define Q4_SK_CW 8
@@ -712,6 +676,42 @@ q4_status run_fp4(const uint8_t* wq, const uint8_t* wsc, const float* wts, int64
                      static_cast<int>(B), out, p.nchunks, p.T, y, ydt, ws_part, ws_count, status);
 }
 
+SkPlan bf16_plan(int64_t out, int64_t in, int64_t B, int sms) {
+    return stream_k_plan(out, in, kF4RT, sms, kF4MinIters, f4_nt(B), TcKind<kKindBF16>::chunk_elems);
+}
+
+template <int NT>
+q4_status run_bf16_tc(const void* W, int64_t out, int64_t in, const void* x, int64_t B, void* y,
+                      void* ws, size_t ws_bytes, cudaStream_t st) {
+    const int dev = current_device();
+    const SkPlan p = bf16_plan(out, in, B, sm_count(dev));
+    if (p.row_tiles > static_cast<int64_t>(kWsCounterBytes / 4)) return Q4_ERR_SHAPE;
+    if (ws_bytes < p.ws_bytes) return Q4_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return Q4_ERR_ALIGNMENT;
+    const size_t smax = static_cast<size_t>(max_smem_optin(dev));
+    int stages = kF4MaxStages;
+    F4Geom geo = f4_geom(NT, 0, stages);
+    while (stages > 2 && geo.total > smax) geo = f4_geom(NT, 0, --stages);
+    if (geo.total > smax) return Q4_ERR_UNSUPPORTED;
+    CUtensorMap tmap_w, tmap_x;
+    constexpr uint32_t kBoxElems = TcKind<kKindBF16>::box_step;  // 64 bf16 = one 128-byte row
+    if (!make_tmap_2d(&tmap_w, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, static_cast<uint64_t>(out),
+                      static_cast<uint64_t>(in), kF4RT, kBoxElems) ||
+        !make_tmap_2d(&tmap_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, static_cast<uint64_t>(B),
+                      static_cast<uint64_t>(in), NT, kBoxElems))
+        return Q4_ERR_CUDA;
+    auto kernel = bf16_gemm_tc_kernel<NT>;
+    if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), false)) return Q4_ERR_CUDA;
+    unsigned* status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
+        return Q4_ERR_CUDA;
+    unsigned* ws_count = reinterpret_cast<unsigned*>(ws);
+    float* ws_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kWsCounterBytes);
+    return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3(kF4Threads), geo.total, 1,
+                     true, st, tmap_w, tmap_x, stages, static_cast<int>(B), out, p.nchunks, p.T,
+                     y, 1, ws_part, ws_count, status);
+}
+
 template <bool NV>
 q4_status dispatch_fp4(const uint8_t* wq, const uint8_t* wsc, const float* wts, int64_t out,
                        int64_t in, const uint8_t* xq, const uint8_t* xsc, const float* xts,
@@ -975,43 +975,26 @@ q4_status q4_gemv_noalloc(const q4_weight* w, const void* x, q4_dtype x_dtype, i
                : dispatch_gemv<false>(w, x, B, y, ydt, scratch, kNoAllocScratchBytes, st);
 }
 
+size_t bf16_ref_workspace_bytes(int64_t out, int64_t in, int64_t B) {
+    if (out <= 0 || in <= 0 || B < 1 || B > 128) return 0;
+    return bf16_plan(out, in, B, sm_count(current_device())).ws_bytes;
+}
+
 q4_status bf16_gemv_ref_bw(const void* W, int64_t out, int64_t in, const void* x, int64_t B,
-                           void* y, q4_stream stream) {
+                           void* y, void* workspace, size_t workspace_bytes, q4_stream stream) {
     if (out < 0 || in <= 0 || (in % 64) != 0) return Q4_ERR_SHAPE;
     if (B < 1 || B > 128) return Q4_ERR_SHAPE;
-    if (in > (int64_t(1) << 30) || out > int64_t(65535) * 128) return Q4_ERR_SHAPE;
     if (out == 0) return Q4_OK;
     if (!W || !x || !y) return Q4_ERR_INVALID_ARG;
     if (!aligned(W, 16) || !aligned(x, 16) || !aligned(y, 16)) return Q4_ERR_ALIGNMENT;
-    if (B > 8) return Q4_ERR_UNSUPPORTED;
+    if (!workspace) return Q4_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const int dev = current_device();
-    const int sms = sm_count(dev);
-    const int nchunks = static_cast<int>(in / kDenseChunkCols);
-    SplitPlan p = plan_split(out, nchunks, kGemvRT, sms);
-    DenseGeom geo = dense_geom(kGemvRT, kGemvStages, p.cps, static_cast<int>(B));
-    const int smax = max_smem_optin(dev);
-    while (geo.total > static_cast<size_t>(smax) && p.S < 16) {
-        p.S = p.S * 2 > 16 ? 16 : p.S * 2;
-        p.cps = (nchunks + p.S - 1) / p.S;
-        p.S = (nchunks + p.cps - 1) / p.cps;
-        geo = dense_geom(kGemvRT, kGemvStages, p.cps, static_cast<int>(B));
-        if (p.S == 16 || p.cps == 1) break;
+    switch (f4_nt(B)) {
+        case 16: return run_bf16_tc<16>(W, out, in, x, B, y, workspace, workspace_bytes, st);
+        case 32: return run_bf16_tc<32>(W, out, in, x, B, y, workspace, workspace_bytes, st);
+        case 64: return run_bf16_tc<64>(W, out, in, x, B, y, workspace, workspace_bytes, st);
+        default: return run_bf16_tc<128>(W, out, in, x, B, y, workspace, workspace_bytes, st);
     }
-    if (geo.total > static_cast<size_t>(smax)) return Q4_ERR_UNSUPPORTED;
-    CUtensorMap tmap;
-    if (!make_tmap_2d(&tmap, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, static_cast<uint64_t>(out),
-                      static_cast<uint64_t>(in), kGemvRT, kDenseChunkCols))
-        return Q4_ERR_CUDA;
-    auto kernel = bf16_gemv_kernel<kGemvMT, kGemvCW, kGemvStages>;
-    if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), p.S > 8)) return Q4_ERR_CUDA;
-    unsigned* status = nullptr;
-    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
-        return Q4_ERR_CUDA;
-    const dim3 grid(p.S, static_cast<unsigned>((out + kGemvRT - 1) / kGemvRT));
-    return launch_cluster(kernel, grid, dim3((kGemvCW + 1) * 32), geo.total, p.S, st, tmap,
-                          reinterpret_cast<const uint16_t*>(x), static_cast<int>(B), out, in,
-                          p.cps, nchunks, y, status);
 }
 
 // ------------------------------------------------- per-channel INT8 weights

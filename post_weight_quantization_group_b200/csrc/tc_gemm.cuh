@@ -1,8 +1,10 @@
-// fp4_gemm.cuh -- W4A4 product of two FP4 microscaling operands on the
-// block-scaled tcgen05 tensor cores of sm_100a.
+// tc_gemm.cuh -- streaming products on the tcgen05 tensor cores of sm_100a
+// whose operands go from HBM to the tensor core without conversion: the
+// W4A4 product of two FP4 microscaling operands (block-scaled MMA) and the
+// unquantised bf16 reference product.
 //
-// "post-training-quantization-gptq-awq-and-rotation" (arganzheng.life),
-// sections 九.1 and 九.2: the weights and the activations both hold E2M1
+// W4A4 ("post-training-quantization-gptq-awq-and-rotation" (arganzheng.life),
+// sections 九.1 and 九.2): the weights and the activations both hold E2M1
 // codes with one scale per small block along K -- an E8M0 power of two per
 // 32 elements (MXFP4) or an E4M3 value per 16 elements under one fp32 scale
 // per tensor (NVFP4).  The product is
@@ -13,6 +15,12 @@
 // applies S_W and S_X inside the tensor core, so the codes go from HBM to the
 // tensor core untouched: no unpacking and no per-group rescale on the CUDA
 // cores (the INT4 kernels spend most of their issue slots there).
+//
+// bf16 reference ("LLM 后训练量化深度实战" (ybb.press) section 一,
+// roofline_bound; arganzheng.life section 二.4, the BF16 vs W4A16 batch
+// table): y = x W^T with fp32 accumulation, the same pipeline with bf16
+// tiles (kind::f16 MMAs, K = 16 per MMA, 128 values of K per stage) and no
+// scale factors.
 //
 // Work decomposition: the persistent stream-K split of the INT4 kernels
 // (q4_gemv_sk.cuh): T = row_tiles x chunks iterations, a row tile is 128 rows
@@ -26,7 +34,7 @@
 //    and the activation codes [NT x 256 B] (each as two 128-byte-swizzled
 //    K-major boxes; activation rows >= B read as zero), and of both operands'
 //    scale bytes [rows x 512/VS] (row-major, as the quantizers write them);
-//  * warps 2-5, scale writers (one per tensor-memory lane quarter): the MMA
+//  * warps 2-5, scale writers (FP4 only; one per tensor-memory lane quarter): the MMA
 //    reads the scale of row m, K-block j from tensor-memory lane m mod 32
 //    (in every lane quarter), column m / 32, byte j -- the 32-lane x 128-bit
 //    pattern replicated four times.  Each warp reads rows lane + 32 i
@@ -61,15 +69,27 @@ constexpr int kF4MaxStages = 4;
 constexpr int kF4Threads = 320;
 constexpr uint32_t kF4TmemCols = 512;
 
-template <bool NV>
-struct F4Fmt {
-    static constexpr int VS = NV ? 16 : 32;                // elements per scale
-    static constexpr int sf_bytes = kF4ChunkCodes / VS;    // scale bytes per row per stage
+// Operand kinds of the streaming tcgen05 product.
+constexpr int kKindMXFP4 = 0;
+constexpr int kKindNVFP4 = 1;
+constexpr int kKindBF16 = 2;
+
+template <int KIND>
+struct TcKind {
+    static constexpr bool fp4 = KIND != kKindBF16;
+    static constexpr bool NV = KIND == kKindNVFP4;
+    static constexpr int VS = NV ? 16 : 32;                       // elements per scale (FP4)
+    static constexpr int chunk_elems = fp4 ? kF4ChunkCodes : 128;  // K per stage (256 B per row)
+    static constexpr int box_step = fp4 ? kF4Box : 64;  // TMA coordinate of one 128-byte box
+    static constexpr int sf_bytes = fp4 ? kF4ChunkCodes / VS : 0;  // scale bytes per row per stage
     // tensor-memory columns of one operand's scales per stage: one column
     // per 32-bit word of a row's scale bytes and per row quarter
     static constexpr int sf_cols = sf_bytes;
     static constexpr uint32_t scale_format = NV ? 0u : 1u;  // E4M3 / E8M0
 };
+
+template <bool NV>
+using F4Fmt = TcKind<NV ? kKindNVFP4 : kKindMXFP4>;
 
 struct F4Geom {
     size_t off_x, off_sw, off_sx, stage_bytes, off_bar, total;
@@ -220,21 +240,26 @@ __device__ __forceinline__ void gather_scales(uint32_t tile, int lane, int nrows
     }
 }
 
-template <bool NV, int NT>
-__global__ void __launch_bounds__(kF4Threads, 1)
-    fp4_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
-                       const __grid_constant__ CUtensorMap tmap_sw,
-                       const __grid_constant__ CUtensorMap tmap_x,
-                       const __grid_constant__ CUtensorMap tmap_sx,
-                       const float* __restrict__ w_ts, const float* __restrict__ x_ts, int stages,
-                       int B, int64_t out, int nchunks, int64_t T, void* __restrict__ y, int ydt,
-                       float* __restrict__ ws_part, unsigned* __restrict__ ws_count,
-                       unsigned* __restrict__ status) {
-    constexpr int SFB = F4Fmt<NV>::sf_bytes;
-    constexpr int SFC = F4Fmt<NV>::sf_cols;
+template <int KIND, int NT>
+__device__ __forceinline__ void tc_gemm_body(const CUtensorMap& tmap_w, const CUtensorMap& tmap_sw,
+                                             const CUtensorMap& tmap_x, const CUtensorMap& tmap_sx,
+                                             const float* __restrict__ w_ts,
+                                             const float* __restrict__ x_ts, int stages, int B,
+                                             int64_t out, int nchunks, int64_t T,
+                                             void* __restrict__ y, int ydt,
+                                             float* __restrict__ ws_part,
+                                             unsigned* __restrict__ ws_count,
+                                             unsigned* __restrict__ status) {
+    using K = TcKind<KIND>;
+    constexpr bool NV = K::NV;
+    constexpr int SFB = K::sf_bytes;
+    constexpr int SFC = K::sf_cols;
+    constexpr int BOX = K::box_step;
     constexpr uint32_t kSf0 = 2 * NT;   // first scale-factor column
-    constexpr uint32_t kIdesc = umma_idesc_f4<NV, NT>();
+    constexpr uint32_t kIdesc =
+        K::fp4 ? umma_idesc_f4<NV, NT>() : umma_idesc_f16<true, kF4RT, NT>();
     constexpr int PW = NT < 32 ? NT : 32;  // accumulator columns per tcgen05.ld
+    constexpr int PF = 16;                 // columns per step of the fix-up
     static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "activation tile width");
     static_assert(2 * NT + kF4MaxStages * 2 * SFC <= static_cast<int>(kF4TmemCols),
                   "tensor memory");
@@ -288,15 +313,17 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         // ------------------------------------------------------ producer
         if (lane == 0 && nit > 0) {
             prefetch_tmap(&tmap_w);
-            prefetch_tmap(&tmap_sw);
             prefetch_tmap(&tmap_x);
-            prefetch_tmap(&tmap_sx);
+            if constexpr (K::fp4) {
+                prefetch_tmap(&tmap_sw);
+                prefetch_tmap(&tmap_sx);
+            }
             const uint32_t tx = (kF4RT + NT) * (kF4ChunkBytes + SFB);
             auto load_w = [&](uint8_t* st, int chunk, int tile, uint64_t* bar) {
-                tma_load_2d(st, &tmap_w, chunk * kF4ChunkBytes, tile * kF4RT, bar);
-                tma_load_2d(st + kF4RT * kF4Box, &tmap_w, chunk * kF4ChunkBytes + kF4Box,
-                            tile * kF4RT, bar);
-                tma_load_2d(st + geo.off_sw, &tmap_sw, chunk * SFB, tile * kF4RT, bar);
+                tma_load_2d(st, &tmap_w, chunk * 2 * BOX, tile * kF4RT, bar);
+                tma_load_2d(st + kF4RT * kF4Box, &tmap_w, chunk * 2 * BOX + BOX, tile * kF4RT, bar);
+                if constexpr (K::fp4)
+                    tma_load_2d(st + geo.off_sw, &tmap_sw, chunk * SFB, tile * kF4RT, bar);
             };
             const int pre = nit < stages ? nit : stages;
             {
@@ -322,10 +349,10 @@ __global__ void __launch_bounds__(kF4Threads, 1)
                     mbar_arrive_expect_tx(&full[s], tx);
                     load_w(st, chunk, tile, &full[s]);
                 }
-                tma_load_2d(st + geo.off_x, &tmap_x, chunk * kF4ChunkBytes, 0, &full[s]);
-                tma_load_2d(st + geo.off_x + NT * kF4Box, &tmap_x, chunk * kF4ChunkBytes + kF4Box,
-                            0, &full[s]);
-                tma_load_2d(st + geo.off_sx, &tmap_sx, chunk * SFB, 0, &full[s]);
+                tma_load_2d(st + geo.off_x, &tmap_x, chunk * 2 * BOX, 0, &full[s]);
+                tma_load_2d(st + geo.off_x + NT * kF4Box, &tmap_x, chunk * 2 * BOX + BOX, 0,
+                            &full[s]);
+                if constexpr (K::fp4) tma_load_2d(st + geo.off_sx, &tmap_sx, chunk * SFB, 0, &full[s]);
                 if (++chunk == nchunks) {
                     chunk = 0;
                     ++tile;
@@ -355,7 +382,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
                     ok = mbar_wait_bounded(&acc_empty[a], static_cast<uint32_t>((seg >> 1) - 1) & 1u,
                                            status, kWaitLimitNs);
                 if (ok) ok = mbar_wait_bounded(&full[s], ph, status, kWaitLimitNs);
-                if (ok) ok = mbar_wait_bounded(&sf_ready[s], ph, status, kWaitLimitNs);
+                if (K::fp4 && ok) ok = mbar_wait_bounded(&sf_ready[s], ph, status, kWaitLimitNs);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t st = sb + static_cast<uint32_t>(geo.stage_bytes) * s;
@@ -368,11 +395,16 @@ __global__ void __launch_bounds__(kF4Threads, 1)
                         st + static_cast<uint32_t>((kk >> 2) * kF4RT * kF4Box) + koff);
                     const uint64_t bd = umma_desc_sw128_kmajor(
                         st + static_cast<uint32_t>(geo.off_x + (kk >> 2) * NT * kF4Box) + koff);
-                    const uint32_t col = NV ? 4u * kk : 4u * (kk >> 1);
-                    const uint32_t sid = NV ? 0u : 2u * (kk & 1);
-                    umma_f4<NV>(tbase + static_cast<uint32_t>(a * NT), ad, bd,
-                                kIdesc | (sid << 29) | (sid << 4), (sfa + col) | (sid << 30),
-                                (sfb + col) | (sid << 30), (seg_first && kk == 0) ? 0u : 1u);
+                    const uint32_t acc = (seg_first && kk == 0) ? 0u : 1u;
+                    if constexpr (K::fp4) {
+                        const uint32_t col = NV ? 4u * kk : 4u * (kk >> 1);
+                        const uint32_t sid = NV ? 0u : 2u * (kk & 1);
+                        umma_f4<NV>(tbase + static_cast<uint32_t>(a * NT), ad, bd,
+                                    kIdesc | (sid << 29) | (sid << 4), (sfa + col) | (sid << 30),
+                                    (sfb + col) | (sid << 30), acc);
+                    } else {
+                        umma_f16_ss(tbase + static_cast<uint32_t>(a * NT), ad, bd, kIdesc, acc);
+                    }
                 }
                 umma_commit(&empty[s]);  // the stage's codes and scales are no longer read
                 const bool seg_end = chunk == nchunks - 1 || c == nit - 1;
@@ -393,6 +425,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         }
     } else if (warp < 6) {
         // ------------------------------------------------ scale writers
+        if constexpr (K::fp4) {
         const uint32_t tl = tbase + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
         const uint32_t sb = smem_u32(smem);
         bool ok = true;
@@ -419,6 +452,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
                 s = 0;
                 ph ^= 1u;
             }
+        }
         }
     } else {
         // ------------------------------------------------------- epilogue
@@ -517,10 +551,10 @@ __global__ void __launch_bounds__(kF4Threads, 1)
                             const bool fs = (T * qq) / P >= t64 * nchunks;
                             const float* src = ws_part + static_cast<size_t>(2 * qq + (fs ? 0 : 1)) *
                                                              kF4RT * NT;
-                            for (int pi = 0; pi < NT / PW; ++pi)
+                            for (int pi = 0; pi < NT / PF; ++pi)
                                 bulk_load_g2s(fix_smem + static_cast<uint32_t>(
-                                                             (pi * nothers + j) * PW * kF4RT * 4),
-                                              src + pi * PW * kF4RT, PW * kF4RT * 4, fixbar);
+                                                             (pi * nothers + j) * PF * kF4RT * 4),
+                                              src + pi * PF * kF4RT, PF * kF4RT * 4, fixbar);
                             ++j;
                         }
                     }
@@ -532,34 +566,34 @@ __global__ void __launch_bounds__(kF4Threads, 1)
                         okf = __all_sync(0xffffffffu, okf);
                         // contributors in CTA order, this CTA's own part from tensor memory
 #pragma unroll 1
-                        for (int pi = 0; pi < NT / PW; ++pi) {
-                            const int c0 = pi * PW;
-                            uint32_t v[PW];
+                        for (int pi = 0; pi < NT / PF; ++pi) {
+                            const int c0 = pi * PF;
+                            uint32_t v[PF];
                             if (okf) {
-                                tmem_ld_cols<PW>(tl + static_cast<uint32_t>(a * NT + c0), v);
+                                tmem_ld_cols<PF>(tl + static_cast<uint32_t>(a * NT + c0), v);
                                 tmem_wait_ld();
                             }
                             if (okf && c0 < B && row < out) {
-                                float acc[PW];
+                                float acc[PF];
 #pragma unroll
-                                for (int e = 0; e < PW; ++e) acc[e] = 0.f;
+                                for (int e = 0; e < PF; ++e) acc[e] = 0.f;
                                 int j = 0;
                                 for (int64_t qq = q_lo; qq <= q_hi; ++qq) {
                                     if (qq == p) {
 #pragma unroll
-                                        for (int e = 0; e < PW; ++e) acc[e] += __uint_as_float(v[e]);
+                                        for (int e = 0; e < PF; ++e) acc[e] += __uint_as_float(v[e]);
                                     } else {
                                         const uint32_t blk =
                                             fix_smem +
-                                            static_cast<uint32_t>(((pi * nothers + j) * PW * kF4RT + r) * 4);
+                                            static_cast<uint32_t>(((pi * nothers + j) * PF * kF4RT + r) * 4);
 #pragma unroll
-                                        for (int e = 0; e < PW; ++e)
+                                        for (int e = 0; e < PF; ++e)
                                             acc[e] += __uint_as_float(lds32(blk + e * kF4RT * 4));
                                         ++j;
                                     }
                                 }
 #pragma unroll
-                                for (int e = 0; e < PW; ++e)
+                                for (int e = 0; e < PF; ++e)
                                     if (c0 + e < B)
                                         store_y(y, ydt, static_cast<int64_t>(c0 + e) * out + row,
                                                 g * acc[e]);
@@ -567,24 +601,24 @@ __global__ void __launch_bounds__(kF4Threads, 1)
                         }
                     } else if (row < out) {
                         // a fix-up while the pipeline still runs: from global
-                        // memory, PW independent loads per contributor
+                        // memory, PF independent loads per contributor
 #pragma unroll 1
-                        for (int c0 = 0; c0 < NT; c0 += PW) {
+                        for (int c0 = 0; c0 < NT; c0 += PF) {
                             if (c0 < B) {
-                                float acc[PW];
+                                float acc[PF];
 #pragma unroll
-                                for (int e = 0; e < PW; ++e) acc[e] = 0.f;
+                                for (int e = 0; e < PF; ++e) acc[e] = 0.f;
                                 for (int64_t qq = q_lo; qq <= q_hi; ++qq) {
                                     const bool fs = (T * qq) / P >= t64 * nchunks;
                                     const int qs = static_cast<int>(2 * qq + (fs ? 0 : 1));
                                     const float* pq =
                                         ws_part + static_cast<size_t>(qs) * kF4RT * NT + r;
 #pragma unroll
-                                    for (int e = 0; e < PW; ++e)
+                                    for (int e = 0; e < PF; ++e)
                                         if (c0 + e < B) acc[e] += __ldcg(pq + (c0 + e) * kF4RT);
                                 }
 #pragma unroll
-                                for (int e = 0; e < PW; ++e)
+                                for (int e = 0; e < PF; ++e)
                                     if (c0 + e < B)
                                         store_y(y, ydt, static_cast<int64_t>(c0 + e) * out + row,
                                                 g * acc[e]);
@@ -607,6 +641,34 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         tc_fence_after();
         tmem_dealloc(tbase, kF4TmemCols);
     }
+}
+
+// W4A4 product of two FP4 operands (NVFP4 or MXFP4).
+template <bool NV, int NT>
+__global__ void __launch_bounds__(kF4Threads, 1)
+    fp4_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                       const __grid_constant__ CUtensorMap tmap_sw,
+                       const __grid_constant__ CUtensorMap tmap_x,
+                       const __grid_constant__ CUtensorMap tmap_sx,
+                       const float* __restrict__ w_ts, const float* __restrict__ x_ts, int stages,
+                       int B, int64_t out, int nchunks, int64_t T, void* __restrict__ y, int ydt,
+                       float* __restrict__ ws_part, unsigned* __restrict__ ws_count,
+                       unsigned* __restrict__ status) {
+    tc_gemm_body<NV ? kKindNVFP4 : kKindMXFP4, NT>(tmap_w, tmap_sw, tmap_x, tmap_sx, w_ts, x_ts,
+                                                   stages, B, out, nchunks, T, y, ydt, ws_part,
+                                                   ws_count, status);
+}
+
+// The bf16 reference product y = x W^T (bf16 W and x, fp32 accumulation).
+template <int NT>
+__global__ void __launch_bounds__(kF4Threads, 1)
+    bf16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                        const __grid_constant__ CUtensorMap tmap_x, int stages, int B, int64_t out,
+                        int nchunks, int64_t T, void* __restrict__ y, int ydt,
+                        float* __restrict__ ws_part, unsigned* __restrict__ ws_count,
+                        unsigned* __restrict__ status) {
+    tc_gemm_body<kKindBF16, NT>(tmap_w, tmap_w, tmap_x, tmap_x, nullptr, nullptr, stages, B, out,
+                                nchunks, T, y, ydt, ws_part, ws_count, status);
 }
 
 }  // namespace q4dev

@@ -124,13 +124,20 @@ def test_product_validation(lib):
 
 
 def test_bf16_reference_and_dequant_validation(lib):
-    f = lib.bf16_gemv_ref_bw
-    assert f(A16, 64, 100, A16, 1, A16, None) == q4.Q4_ERR_SHAPE      # in not multiple of 64
-    assert f(A16, 64, 128, A16, 0, A16, None) == q4.Q4_ERR_SHAPE
-    assert f(A16, 64, 128, A16, 129, A16, None) == q4.Q4_ERR_SHAPE
-    assert f(None, 64, 128, A16, 1, A16, None) == q4.Q4_ERR_INVALID_ARG
-    assert f(A2, 64, 128, A16, 1, A16, None) == q4.Q4_ERR_ALIGNMENT
-    assert f(A16, 0, 128, A16, 1, A16, None) == q4.Q4_OK
+    def f(W=A16, out=64, inn=128, x=A16, B=1, y=A16, ws=A16):
+        return lib.bf16_gemv_ref_bw(W, out, inn, x, B, y, ws, 1 << 24, None)
+
+    assert f(inn=100) == q4.Q4_ERR_SHAPE      # in not multiple of 64
+    assert f(B=0) == q4.Q4_ERR_SHAPE
+    assert f(B=129) == q4.Q4_ERR_SHAPE
+    assert f(W=None) == q4.Q4_ERR_INVALID_ARG
+    assert f(W=A2) == q4.Q4_ERR_ALIGNMENT
+    assert f(y=A16 + 2) == q4.Q4_ERR_ALIGNMENT
+    assert f(ws=None) == q4.Q4_ERR_WORKSPACE
+    assert f(out=0) == q4.Q4_OK
+    assert lib.bf16_ref_workspace_bytes(64, 128, 0) == 0
+    assert lib.bf16_ref_workspace_bytes(64, 128, 129) == 0
+    assert lib.bf16_ref_workspace_bytes(64, 128, 128) > 0
     d = lib.q4_dequant
     assert d(ctypes.byref(_w()), None, q4.Q4_F32, None) == q4.Q4_ERR_INVALID_ARG
     assert d(ctypes.byref(_w()), A16, 5, None) == q4.Q4_ERR_INVALID_ARG

@@ -257,14 +257,20 @@ def test_gemv_empty_and_bad_alignment():
 
 # ------------------------------------------------------ bf16 reference GEMV
 
-@pytest.mark.parametrize("shape", [(300, 1024), (4096, 4096), (8192, 28672), (14336, 4096)])
-@pytest.mark.parametrize("B", [1, 4, 8])
+@pytest.mark.parametrize("shape", [(300, 1024), (4096, 4096), (8192, 28672), (14336, 4096),
+                                   (200, 1088)])
+@pytest.mark.parametrize("B", [1, 4, 8, 9, 16, 33, 64, 128])
 def test_bf16_reference(shape, B):
+    """Row tiles split between CTAs (8192 x 28672), whole tiles (14336 x
+    4096), a ragged row tile and a K tail inside a chunk (200 x 1088), every
+    activation tile width."""
     out, inn = shape
     W = wl.normal_weight(out, inn, 30, device="cuda").to(torch.bfloat16)
     x = wl.activations(B, inn, 31, device="cuda")
     y = q4.bf16_gemv_ref_bw(W, x)
     torch.cuda.synchronize()
+    assert q4.q4_sync_status() == q4.Q4_OK
+    assert torch.equal(q4.bf16_gemv_ref_bw(W, x), y)  # deterministic
     rows = _sample_rows(out, 128)
     Wr = _f32(W[torch.as_tensor(rows, device="cuda")])
     y_ref = oracle.dense(Wr, x.float().cpu().numpy().astype(np.float64))
