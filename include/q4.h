@@ -229,11 +229,18 @@ Q4_API q4_status q4_gemv(const q4_weight* w, const void* x, q4_dtype x_dtype, in
 /*
  * The same product for batches 1 <= B <= 128 (the skinny-GEMM regime of
  * arganzheng.life section 二.4, where W4A16 turns compute-bound near
- * B = ridge / 4).  B <= 8 runs the q4_gemv kernel; 9 <= B <= 128 runs on the
+ * B = ridge / 4).  B <= 8 runs the q4_gemv kernel; 9 <= B <= 64 runs on the
  * tcgen05 tensor cores: codes unpacked to exact 16-bit integers in tensor
- * memory, activations padded to 16/32/64/128 columns, fp32 accumulation per
- * group, group partials scaled in fp32.  Same arguments and requirements as
- * q4_gemv (the workspace of q4_workspace_bytes for this B), same tolerance,
+ * memory, activations padded to 16/32/64 columns, fp32 accumulation per
+ * group, group partials scaled in fp32.  65 <= B <= 128 runs on the tcgen05
+ * tensor cores with the group scale applied while unpacking: each weight
+ * becomes fp16(s * (q - z)) (one fp16 rounding, relative error <= 2^-11),
+ * the activations are taken in fp16 (bf16 ones are converted first, into the
+ * workspace), and one fp32 accumulator spans the whole K range; an
+ * activation of magnitude above 65504 (fp16's largest finite value) is then
+ * reported by q4_sync_status as Q4_ERR_INVALID_ARG.  Same arguments and
+ * requirements as q4_gemv (the workspace of q4_workspace_bytes for this B,
+ * which for B > 64 includes room for the fp16 activations), same tolerance,
  * bit-for-bit reproducible.
  */
 Q4_API q4_status q4_gemm_skinny(const q4_weight* w, const void* x, q4_dtype x_dtype, int64_t B,

@@ -1,7 +1,7 @@
 // q4_api.cu -- the C ABI of include/q4.h: argument validation, launch
 // planning, TMA descriptor encoding and kernel launches.  All kernels live in
 // this translation unit (q4_quant.cuh, q4_gemv.cuh, q4_gemv_sk.cuh,
-// q4_skinny_tc.cuh, q8_gemv.cuh, q8_quant.cuh, fp4_quant.cuh, tc_gemm.cuh).
+// q4_skinny_tc.cuh, q4_skinny_f16.cuh, q8_gemv.cuh, q8_quant.cuh, fp4_quant.cuh, tc_gemm.cuh).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -18,6 +18,7 @@
 #include "q4_gemv_sk.cuh"
 #include "q4_quant.cuh"
 #include "q4_skinny_tc.cuh"
+#include "q4_skinny_f16.cuh"
 #include "q8_gemv.cuh"
 #include "q8_quant.cuh"
 #include "fp4_quant.cuh"
@@ -289,8 +290,12 @@ int tc_ctas_per_sm(int nt) { return nt <= 32 ? 2 : 1; }
 
 SkPlan tc_plan(int64_t out, int64_t in, int64_t B, int sms) {
     const int nt = tc_nt(B);
-    return stream_k_plan(out, in, kTcRT, static_cast<int64_t>(tc_ctas_per_sm(nt)) * sms,
-                         kTcMinIters, nt);
+    SkPlan p = stream_k_plan(out, in, kTcRT, static_cast<int64_t>(tc_ctas_per_sm(nt)) * sms,
+                             kTcMinIters, nt);
+    // NT = 128 runs the scaled-fp16 kernel, whose bf16 activations are first
+    // converted to fp16 into the workspace, after the partial slots
+    if (nt == 128) p.ws_bytes += align_up(static_cast<size_t>(B) * in * 2, 256);
+    return p;
 }
 
 SkPlan product_plan(int64_t out, int64_t in, int64_t B, int sms) {
@@ -501,14 +506,95 @@ q4_status run_skinny(const q4_weight* w, const void* x, int64_t B, void* y, int 
                      status);
 }
 
+// The scaled-fp16 tcgen05 kernel (q4_skinny_f16.cuh) for NT = 128; bf16
+// activations are converted to fp16 first, into the workspace.
+template <bool BF16, int GS, int NT>
+q4_status run_skinny_f16(const q4_weight* w, const void* x, int64_t B, void* y, int ydt, void* ws,
+                         size_t ws_bytes, cudaStream_t st) {
+    const int dev = current_device();
+    const SkPlan p = tc_plan(w->out, w->in, B, sm_count(dev));
+    if (!ws || ws_bytes < p.ws_bytes) return Q4_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return Q4_ERR_ALIGNMENT;
+    const bool sym = w->symmetric != 0;
+    constexpr int cps = F16Cfg<NT>::ctas_per_sm;
+    const size_t per_sm = 228 * 1024;
+    const size_t smax = static_cast<size_t>(max_smem_optin(dev));
+    int stages = kTcMaxStages;
+    TcGeom geo = tc_geom(NT, stages, sym);
+    while (stages > 2 && (cps * (geo.total + 1024) > per_sm || geo.total > smax)) {
+        --stages;
+        geo = tc_geom(NT, stages, sym);
+    }
+    if (cps * (geo.total + 1024) > per_sm || geo.total > smax) return Q4_ERR_UNSUPPORTED;
+    const int64_t G = w->in / GS;
+    const bool meta_tma = (G % 8) == 0 && aligned(w->scales, 16) && (sym || aligned(w->zeros, 16));
+    CUtensorMap tmap_w, tmap_x, tmap_s, tmap_z;
+    std::memset(&tmap_s, 0, sizeof(tmap_s));
+    std::memset(&tmap_z, 0, sizeof(tmap_z));
+    if (!make_tmap_2d(&tmap_w, w->qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                      static_cast<uint64_t>(w->out), static_cast<uint64_t>(w->in / 2), kTcRT,
+                      kChunkBytes))
+        return Q4_ERR_CUDA;
+    unsigned* status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
+        return Q4_ERR_CUDA;
+    const void* xf = x;
+    if (BF16) {
+        void* xw = reinterpret_cast<uint8_t*>(ws) + kWsCounterBytes + p.ws_part_bytes;
+        const int64_t n8 = B * w->in / 8;
+        const int blocks = static_cast<int>(std::min<int64_t>((n8 + 255) / 256, 4LL * sm_count(dev)));
+        const q4_status s0 = launch_ex(x_to_f16_kernel, dim3(static_cast<unsigned>(blocks)),
+                                       dim3(256), 0, 1, true, st,
+                                       reinterpret_cast<const uint4*>(x), n8,
+                                       reinterpret_cast<uint4*>(xw), status);
+        if (s0 != Q4_OK) return s0;
+        xf = xw;
+    }
+    if (!make_tmap_2d(&tmap_x, xf, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, static_cast<uint64_t>(B),
+                      static_cast<uint64_t>(w->in), NT, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return Q4_ERR_CUDA;
+    if (meta_tma) {
+        if (!make_tmap_2d(&tmap_s, w->scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                          static_cast<uint64_t>(w->out), static_cast<uint64_t>(G), kTcRT, 8,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+            return Q4_ERR_CUDA;
+        if (!sym && !make_tmap_2d(&tmap_z, w->zeros, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                                  static_cast<uint64_t>(w->out), static_cast<uint64_t>(G), kTcRT,
+                                  8, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return Q4_ERR_CUDA;
+    }
+    auto kernel = q4_skinny_f16_kernel<GS, NT>;
+    if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), false)) return Q4_ERR_CUDA;
+    unsigned* ws_count = reinterpret_cast<unsigned*>(ws);
+    float* ws_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kWsCounterBytes);
+    return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3(F16Cfg<NT>::threads),
+                     geo.total, 1, true, st, tmap_w, tmap_x, tmap_s, tmap_z, meta_tma ? 1 : 0,
+                     reinterpret_cast<const uint16_t*>(w->scales),
+                     reinterpret_cast<const uint16_t*>(w->zeros), sym ? 1 : 0, stages,
+                     static_cast<int>(B), w->out, w->in, p.nchunks, p.T, y, ydt, ws_part, ws_count,
+                     status);
+}
+
 template <bool BF16, int NT>
 q4_status dispatch_skinny_nt(const q4_weight* w, const void* x, int64_t B, void* y, int ydt,
                              void* ws, size_t wsb, cudaStream_t st) {
-    switch (w->group_size) {
-        case 32: return run_skinny<BF16, 32, NT>(w, x, B, y, ydt, ws, wsb, st);
-        case 64: return run_skinny<BF16, 64, NT>(w, x, B, y, ydt, ws, wsb, st);
-        case 128: return run_skinny<BF16, 128, NT>(w, x, B, y, ydt, ws, wsb, st);
-        default: return Q4_ERR_UNSUPPORTED;
+    // B > 64: the scales go into the fp16 A operand and one accumulator
+    // covers a segment (the exact kernel's per-group rescale of 128 columns
+    // bounds it there); B <= 64: exact codes, per-group rescale
+    if constexpr (NT == 128) {
+        switch (w->group_size) {
+            case 32: return run_skinny_f16<BF16, 32, NT>(w, x, B, y, ydt, ws, wsb, st);
+            case 64: return run_skinny_f16<BF16, 64, NT>(w, x, B, y, ydt, ws, wsb, st);
+            case 128: return run_skinny_f16<BF16, 128, NT>(w, x, B, y, ydt, ws, wsb, st);
+            default: return Q4_ERR_UNSUPPORTED;
+        }
+    } else {
+        switch (w->group_size) {
+            case 32: return run_skinny<BF16, 32, NT>(w, x, B, y, ydt, ws, wsb, st);
+            case 64: return run_skinny<BF16, 64, NT>(w, x, B, y, ydt, ws, wsb, st);
+            case 128: return run_skinny<BF16, 128, NT>(w, x, B, y, ydt, ws, wsb, st);
+            default: return Q4_ERR_UNSUPPORTED;
+        }
     }
 }
 
@@ -1295,7 +1381,7 @@ q4_status q4_sync_status(q4_stream stream) {
             noalloc_mark_reclear();
             return Q4_ERR_TIMEOUT;
         }
-        if (h & kStatusBadIndex) return Q4_ERR_INVALID_ARG;
+        if (h & (kStatusBadIndex | kStatusRange)) return Q4_ERR_INVALID_ARG;
     }
     return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }

@@ -13,8 +13,9 @@ namespace q4dev {
 // ---------------------------------------------------------------- status
 // Device-side error word: bit 0 = a bounded wait ran out.
 // Bit 1 = an index argument (a column permutation) was out of range; the
-// kernel clamped it and went on.
-enum : unsigned { kStatusTimeout = 1u, kStatusBadIndex = 2u };
+// kernel clamped it and went on.  Bit 2 = an activation outside fp16's
+// finite range reached a product that takes its activations in fp16.
+enum : unsigned { kStatusTimeout = 1u, kStatusBadIndex = 2u, kStatusRange = 4u };
 
 // A bounded wait gives up after this many nanoseconds (%globaltimer), sets
 // kStatusTimeout in the status word and lets the kernel finish without

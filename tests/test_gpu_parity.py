@@ -553,3 +553,23 @@ def test_act_order_bad_index_is_reported():
 def test_gemv_fused_qkv_and_gate_up_shapes(shape):
     """The Llama-3-8B q/k/v and gate/up matrices stored row-concatenated."""
     _gemv_case(*shape, 128, True, 1, torch.bfloat16, seed=40, rows=_sample_rows(shape[0], 160))
+
+
+@pytest.mark.gpu
+def test_skinny_fp16_activation_range_reported():
+    """B > 64 takes its activations in fp16: a finite bf16 activation beyond
+    fp16's range is reported (Q4_ERR_INVALID_ARG), and the next call with
+    in-range activations is clean and correct."""
+    W = wl.normal_weight(256, 1024, 50, device="cuda")
+    w = q4.q4_quantize_pack(W, 128, True)
+    x = wl.activations(80, 1024, 51, device="cuda")
+    x_big = x.clone()
+    x_big[3, 17] = 1.0e5
+    q4.q4_gemm_skinny(w, x_big)
+    assert q4.q4_sync_status() == q4.Q4_ERR_INVALID_ARG
+    y = q4.q4_gemm_skinny(w, x, y_dtype=torch.float32)
+    assert q4.q4_sync_status() == q4.Q4_OK
+    q_ref, s_ref, z_ref = oracle.quantize_pack(_f32(W), 128, True)
+    y_ref = oracle.gemv(q_ref, s_ref, z_ref, 256, 1024, 128, True,
+                        x.float().cpu().numpy().astype(np.float64))
+    _assert_within(y.cpu().numpy(), y_ref, "skinny B=80 after a range error")
