@@ -11,6 +11,7 @@
 #include <cstring>
 #include <mutex>
 #include <utility>
+#include <vector>
 
 #include "q4.h"
 #include "q4_device.cuh"
@@ -283,6 +284,56 @@ SkPlan sk_plan(int64_t out, int64_t in, int sms) {
     return stream_k_plan(out, in, kSkRT, static_cast<int64_t>(kSkCtasPerSm) * sms, kSkMinIters, 8);
 }
 
+// Cluster fix-up of the B <= 8 kernel.  With P = row_tiles x S the stream-K
+// split gives CTA p the K part p % S of row tile p / S, so the S CTAs of a
+// tile are one aligned cluster: they add their partial tiles through
+// distributed shared memory instead of the workspace, counter and
+// last-arriver pass.  Taken with the largest S <= 8 whose clusters the
+// device holds all at once, unless its CTAs run more than kSkClusterSlack
+// chunks beyond the longest stream-K range; otherwise stream-K.
+#ifndef Q4_SK_CLUSTER_SLACK
+#define Q4_SK_CLUSTER_SLACK 1
+#endif
+constexpr int kSkClusterSlack = Q4_SK_CLUSTER_SLACK;
+
+// Clusters of `s` CTAs of `kernel` resident at once on the current device
+// (cached per kernel, cluster size and shared-memory size; 0 if the query
+// fails, which leaves the caller on stream-K).
+template <typename K>
+int max_active_clusters(K kernel, int s, dim3 block, size_t smem) {
+    struct Entry {
+        const void* k;
+        int dev, s;
+        size_t smem;
+        int n;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> cache;
+    const int dev = current_device();
+    const void* key = reinterpret_cast<const void*>(kernel);
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& e : cache)
+        if (e.k == key && e.dev == dev && e.s == s && e.smem == smem) return e.n;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(s));
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = s;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+    }
+    cache.push_back({key, dev, s, smem, n});
+    return n;
+}
+
 // Skinny-GEMM (tcgen05) kernel: activation tile width NT per batch size.
 constexpr int kTcMinIters = 4;
 int tc_nt(int64_t B) { return B <= 16 ? 16 : B <= 32 ? 32 : B <= 64 ? 64 : 128; }
@@ -327,14 +378,38 @@ q4_status run_gemv(const q4_weight* const* wv, int n, const void* x, int64_t B, 
     // owns fixed slots), so the ring is cut to an even depth.
     const int per_sm = 228 * 1024;
     int stages = kSkMaxStages;
-    SkGeom geo = sk_geom(kSkRT, stages, static_cast<int>(B), SYM);
+    SkGeom geo = sk_geom(kSkRT, stages, static_cast<int>(B), SYM, false);
     while (stages > 2 && kSkCtasPerSm * (geo.total + 1024) > static_cast<size_t>(per_sm)) {
         --stages;
-        geo = sk_geom(kSkRT, stages, static_cast<int>(B), SYM);
+        geo = sk_geom(kSkRT, stages, static_cast<int>(B), SYM, false);
     }
     const bool two_helpers = B >= 4;
-    if (two_helpers && (stages & 1)) geo = sk_geom(kSkRT, --stages, static_cast<int>(B), SYM);
+    if (two_helpers && (stages & 1)) geo = sk_geom(kSkRT, --stages, static_cast<int>(B), SYM, false);
     const int helpers = two_helpers ? 2 : 1;
+    const dim3 block((kSkCW + 1 + helpers) * 32);
+    auto kernel = two_helpers ? q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 2, false>
+                              : q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 1, false>;
+    // the cluster fix-up, when its clusters fit (see kSkClusterSlack)
+    int cluster_s = 1;
+    {
+        const SkGeom gcl = sk_geom(kSkRT, stages, static_cast<int>(B), SYM, true);
+        auto kcl = two_helpers ? q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 2, true>
+                               : q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 1, true>;
+        const int64_t pmax = static_cast<int64_t>(kSkCtasPerSm) * sm_count(dev);
+        const int64_t sk_iters = (p.T + p.P - 1) / p.P;
+        const bool fits = kSkCtasPerSm * (gcl.total + 1024) <= static_cast<size_t>(per_sm);
+        for (int S = 8; fits && S >= 2 && cluster_s == 1; --S) {
+            if (S > p.nchunks || p.row_tiles * S > pmax) continue;
+            if ((p.nchunks + S - 1) / S > sk_iters + kSkClusterSlack) break;
+            if (!set_kernel_attrs(kcl, static_cast<int>(gcl.total), false)) return Q4_ERR_CUDA;
+            if (max_active_clusters(kcl, S, block, gcl.total) >= p.row_tiles) {
+                cluster_s = S;
+                kernel = kcl;
+                geo = gcl;
+            }
+        }
+    }
+    const int64_t grid = cluster_s > 1 ? p.row_tiles * cluster_s : p.P;
     const int64_t G = in / GS;
     // scale / zero windows by TMA when every product's rows are 16-byte aligned
     bool meta_tma = (G % 8) == 0;
@@ -367,17 +442,15 @@ q4_status run_gemv(const q4_weight* const* wv, int n, const void* x, int64_t B, 
                       static_cast<uint64_t>(B), static_cast<uint64_t>(in),
                       static_cast<uint32_t>(B), kChunkCodes, CU_TENSOR_MAP_SWIZZLE_NONE))
         return Q4_ERR_CUDA;
-    auto kernel = two_helpers ? q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 2>
-                              : q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 1>;
     if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), false)) return Q4_ERR_CUDA;
     unsigned* status = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
         return Q4_ERR_CUDA;
     unsigned* ws_count = reinterpret_cast<unsigned*>(ws);
     float* ws_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kWsCounterBytes);
-    return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3((kSkCW + 1 + helpers) * 32),
-                     geo.total, 1, true, st, grp, tmap_x, meta_tma ? 1 : 0, stages,
-                     static_cast<int>(B), in, p.nchunks, p.T, ydt, ws_part, ws_count, status);
+    return launch_ex(kernel, dim3(static_cast<unsigned>(grid)), block, geo.total, cluster_s, true,
+                     st, grp, tmap_x, meta_tma ? 1 : 0, stages, static_cast<int>(B), in,
+                     p.nchunks, p.T, ydt, ws_part, ws_count, status, cluster_s);
 }
 
 template <bool BF16>

@@ -82,7 +82,7 @@ __device__ __forceinline__ int sk_product(const SkGroup& g, int64_t tile) {
 struct SkGeom {
     size_t w_bytes, off_m, m_bytes;              // weight tiles, per-stage slots
     size_t off_x, off_xp, off_sx, off_sc, off_zc;  // inside a per-stage slot
-    size_t off_bar, total;
+    size_t off_bar, off_red, total;
 };
 
 // All stages' weight tiles [rt x 128 B] first (each 1024-byte aligned for
@@ -90,7 +90,7 @@ struct SkGeom {
 // rewritten in place by the helper into MMA fragment order [8 slots x 8
 // batch x 4 threads x 16 B] | group sums [8 groups x 8 batch] fp32 | scale
 // window [rt x 8] fp16 | zero-point window [rt x 8] fp16 (asymmetric only).
-__host__ __device__ inline SkGeom sk_geom(int rt, int stages, int b, bool sym) {
+__host__ __device__ inline SkGeom sk_geom(int rt, int stages, int b, bool sym, bool cluster) {
     SkGeom g{};
     (void)b;  // the activation area is 8 x 512 B for every b <= 8
     g.w_bytes = static_cast<size_t>(rt) * kChunkBytes;
@@ -102,8 +102,16 @@ __host__ __device__ inline SkGeom sk_geom(int rt, int stages, int b, bool sym) {
     g.off_zc = g.off_sc + static_cast<size_t>(rt) * 16;
     g.m_bytes = align_up(g.off_zc + (sym ? 0 : static_cast<size_t>(rt) * 16), 128);
     g.off_bar = align_up(g.off_m + g.m_bytes * stages, 8);
-    g.total = g.off_bar + static_cast<size_t>(3 * kSkMaxStages) * 8 + 64 + 1024;
+    // with the cluster fix-up: the partial tile the cluster reduces through
+    // distributed shared memory
+    g.off_red = align_up(g.off_bar + static_cast<size_t>(3 * kSkMaxStages) * 8 + 64, 16);
+    g.total = g.off_red + (cluster ? static_cast<size_t>(rt) * 8 * 4 : 0) + 1024;
     return g;
+}
+
+// The two cluster barriers of the reduction, for warps with no part in it.
+__device__ __forceinline__ void cluster_idle(int n) {
+    for (int i = 0; i < n; ++i) cluster_sync_all();
 }
 
 // CTA that owns iteration i of T split over P CTAs: it_beg(q) = T q / P.
@@ -127,12 +135,13 @@ __device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v
 // larger batches split the chunks between two helpers (chunk c to helper
 // c % 2).  NH is a template parameter so that each variant gets the register
 // budget of its own block size.
-template <bool BF16, int GS, bool SYM, int CW, int NH>
+template <bool BF16, int GS, bool SYM, int CW, int NH, bool CLUSTER>
 __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
     q4_gemv_sk_kernel(const __grid_constant__ SkGroup grp,
                       const __grid_constant__ CUtensorMap tmap_x, int meta_tma, int stages, int B,
                       int64_t in, int nchunks, int64_t T, int ydt, float* __restrict__ ws_part,
-                      unsigned* __restrict__ ws_count, unsigned* __restrict__ status) {
+                      unsigned* __restrict__ ws_count, unsigned* __restrict__ status,
+                      int cluster_s) {
     constexpr int RT = CW * 16;
     constexpr int GPC = kChunkCodes / GS;  // groups per chunk
     constexpr int WPG = GS / 32;           // 32-bit words per thread per row per group
@@ -141,7 +150,7 @@ __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const SkGeom geo = sk_geom(RT, stages, B, SYM);
+    const SkGeom geo = sk_geom(RT, stages, B, SYM, CLUSTER);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + geo.off_bar);
     uint64_t* sxful = full + kSkMaxStages;
     uint64_t* empty = sxful + kSkMaxStages;
@@ -234,6 +243,7 @@ __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
             }
         }
         __syncwarp();
+        if constexpr (CLUSTER) cluster_idle(2);
         return;
     }
 
@@ -255,7 +265,10 @@ __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
         // k-1 as done.  So nh divides the ring depth; otherwise one helper.
         const int hw = warp - (CW + 1);
         const int nh = stages % NH == 0 ? NH : 1;
-        if (hw >= nh) return;
+        if (hw >= nh) {
+            if constexpr (CLUSTER) cluster_idle(2);
+            return;
+        }
         grid_dependency_wait();
         int tile = tile0, chunk = chunk0, s = 0;
         uint32_t ph = 0;
@@ -348,6 +361,8 @@ __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
                 ph ^= 1u;
             }
         }
+        __syncwarp();
+        if constexpr (CLUSTER) cluster_idle(2);
         return;
     }
 
@@ -472,6 +487,16 @@ __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
                     const int64_t row = row0 + R0 + ((e >> 1) ? 8 : 0);
                     if (col < B && row < out) store_y(y, ydt, static_cast<int64_t>(col) * out + row, acc[e]);
                 }
+            } else if constexpr (CLUSTER) {
+                // the CTA's one segment: its partial tile stays in shared
+                // memory for the cluster's reduction after the loop
+                float* red = reinterpret_cast<float*>(smem + geo.off_red);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int col = 2 * t + (e & 1);
+                    const int row = R0 + ((e >> 1) ? 8 : 0);
+                    red[row * 8 + col] = acc[e];
+                }
             } else {
                 // partial tile: slot 2p (the range's first segment) or 2p + 1
                 const int slot = static_cast<int>(2 * p + (seg_start == 0 ? 0 : 1));
@@ -538,6 +563,31 @@ __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
             s = 0;
             ph ^= 1u;
         }
+    }
+    if constexpr (CLUSTER) {
+        // The S CTAs of a cluster share one row tile (rank r holds K range r
+        // of S): rank r adds rows [RT r / S, RT (r+1) / S) of the S partial
+        // tiles in rank order through distributed shared memory and writes y.
+        __syncwarp();
+        cluster_sync_all();  // every rank's partial tile is in its shared memory
+        const int S = cluster_s;
+        const int r = static_cast<int>(cluster_ctarank());
+        const int pi = sk_product(grp, tile0);
+        const int64_t out = grp.out[pi];
+        void* const y = grp.y[pi];
+        const int64_t row0 = (static_cast<int64_t>(tile0) - grp.tile_beg[pi]) * RT;
+        const uint32_t red = smem_u32(smem + geo.off_red);
+        const int v_end = (RT * (r + 1) / S) * 8;
+        for (int v = (RT * r / S) * 8 + static_cast<int>(threadIdx.x); v < v_end; v += CW * 32) {
+            const int row = v >> 3, col = v & 7;
+            float sum = 0.f;
+            for (int q = 0; q < S; ++q)
+                sum += ld_shared_cluster_f32(mapa_shared(red + static_cast<uint32_t>(v) * 4, q));
+            if (col < B && row0 + row < out)
+                store_y(y, ydt, static_cast<int64_t>(col) * out + row0 + row, sum);
+        }
+        __syncwarp();
+        cluster_sync_all();  // no rank leaves while another still reads it
     }
 }
 

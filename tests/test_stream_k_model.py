@@ -115,3 +115,68 @@ def test_owner_formula_is_the_inverse_of_the_split():
             for p in range(P):
                 for i in range(starts[p], starts[p + 1]):
                     assert owner(i, T, P) == p
+
+
+# ---------------------------------------------------------------- clusters
+# The B <= 8 kernel's cluster fix-up: P = row_tiles x S, and the S CTAs of
+# each row tile (one aligned cluster, rank = p % S) add their partial tiles
+# through distributed shared memory.  The kernel relies on every CTA's range
+# being one non-empty partial segment of row tile p // S, the ranks of a tile
+# covering its chunks in rank order.
+
+def cluster_size(tiles, nchunks, P, pmax, slack=1):
+    """The library's candidate: the largest S <= 8 that fits the grid, unless
+    its CTAs run more than `slack` chunks beyond the longest stream-K range.
+    (On the device it is then taken only if all row_tiles clusters of S CTAs
+    are resident at once, else the next smaller S is tried.)"""
+    T = tiles * nchunks
+    sk_iters = -(-T // P)
+    for S in range(8, 1, -1):
+        if S > nchunks or tiles * S > pmax:
+            continue
+        return S if -(-nchunks // S) <= sk_iters + slack else 1
+    return 1
+
+
+def check_cluster_plan(tiles, nchunks, S):
+    T, P = tiles * nchunks, tiles * S
+    covered = [0] * T
+    for p in range(P):
+        segs = segments(p, T, P, nchunks)
+        assert len(segs) == 1  # one segment: one slot of shared memory
+        tile, chunk, n, _ = segs[0]
+        assert tile == p // S and n >= 1
+        assert not (chunk == 0 and n == nchunks)  # never a whole tile
+        for i in range(tile * nchunks + chunk, tile * nchunks + chunk + n):
+            covered[i] += 1
+        if p % S:  # ranks follow each other along K
+            prev = segments(p - 1, T, P, nchunks)[0]
+            assert prev[0] == tile and prev[1] + prev[2] == chunk
+    assert covered == [1] * T
+
+
+@pytest.mark.parametrize("name,out,inn", SHAPES)
+def test_cluster_plans_launched(name, out, inn):
+    tiles, nchunks = -(-out // 128), -(-inn // 256)
+    P = stream_k_P(tiles * nchunks, 296, 2)
+    S = cluster_size(tiles, nchunks, P, 296)
+    if S > 1:
+        check_cluster_plan(tiles, nchunks, S)
+
+
+def test_cluster_choice_on_the_8b_layer():
+    # q/k/v grouped (48 tiles x 16 chunks), o (32 x 16), down (32 x 56):
+    # cluster candidates; gate/up grouped (224 tiles) keeps stream-K
+    assert cluster_size(48, 16, 296, 296) == 6
+    assert cluster_size(32, 16, 256, 296) == 8
+    assert cluster_size(32, 56, 296, 296) == 8
+    assert cluster_size(224, 16, 296, 296) == 1
+
+
+def test_random_cluster_plans():
+    rng = random.Random(11)
+    for _ in range(300):
+        S = rng.randint(2, 8)
+        nchunks = rng.randint(S, 80)
+        tiles = rng.randint(1, 296 // S)
+        check_cluster_plan(tiles, nchunks, S)
