@@ -385,6 +385,11 @@ q4_status run_gemv(const q4_weight* const* wv, int n, const void* x, int64_t B, 
     }
     const bool two_helpers = B >= 4;
     if (two_helpers && (stages & 1)) geo = sk_geom(kSkRT, --stages, static_cast<int>(B), SYM, false);
+    // TMA destinations: weight tiles 1024-byte aligned (128-byte swizzle),
+    // the activation chunk and the scale / zero-point windows 128-byte aligned
+    if (geo.w_bytes % 1024 || geo.off_m % 1024 || geo.m_bytes % 128 || geo.off_x % 128 ||
+        geo.off_sc % 128 || geo.off_zc % 128)
+        return Q4_ERR_CUDA;
     const int helpers = two_helpers ? 2 : 1;
     const dim3 block((kSkCW + 1 + helpers) * 32);
     auto kernel = two_helpers ? q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 2, false>
