@@ -748,7 +748,8 @@ def run_ours(args):
                      "traffic_unit": "DRAM bytes per launch",
                      "traffic_note": (f"{GEMV_TRAFFIC_RATIO:.4f} x the algorithmic bytes: "
                                       + GEMV_TRAFFIC_SOURCE),
-                     "kernel": "q4_gemv_sk_kernel<bf16,g128,sym,8,1>",
+                     "kernel": ("q4_gemv_sk_kernel<bf16,g128,sym,8,1>: stream-K fix-up for "
+                                "gate/up, cluster fix-up for q/k/v, o and down"),
                      "bytes_per_launch_avg": step_bytes // launches_per_step},
         "clocks": clocks,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
