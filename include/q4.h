@@ -217,6 +217,10 @@ Q4_API size_t q4_workspace_bytes(int64_t out, int64_t in, int64_t B, int32_t gro
  *              of any shape in stream order.  Calls that may overlap on the
  *              GPU need separate buffers.  After a call that ends in
  *              Q4_ERR_TIMEOUT, re-zero it.
+ * Small products (row tiles x S CTAs fit the device, S <= 8) split each
+ * 128-row tile's K range over a thread-block cluster of S CTAs that add
+ * their partials through distributed shared memory; those launches leave the
+ * workspace untouched.  The plan depends only on the shape and the device.
  * The K reduction order is fixed, so results are bit-for-bit reproducible.
  * Summation order differs from the fp64 oracle; results agree within
  * |y - y_ref| <= 4e-3 * (|y_ref| + rms(y_ref)) (the bf16 output rounding
