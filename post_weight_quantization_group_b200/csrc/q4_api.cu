@@ -296,6 +296,16 @@ SkPlan sk_plan(int64_t out, int64_t in, int sms) {
 #endif
 constexpr int kSkClusterSlack = Q4_SK_CLUSTER_SLACK;
 
+// Whole-tile grid of the B <= 8 kernel: when the row tiles alone nearly fill
+// the grid (and no cluster plan is taken), one CTA per row tile has no
+// partial tile and no fix-up at all.  Stream-K's shorter ranges pay two
+// partial-tile epilogues per CTA (partial stores, counter atomic, the last
+// arriver's reads), measured at about four chunks' worth of time per CTA; so
+// the whole-tile grid is taken when it costs at most kSkWholeTileSlack chunks
+// over the longest stream-K range (8B gate/up, 224 tiles x 16 chunks: 18.5
+// against 20.2 us; 70B gate, 224 x 32 chunks, 7 more: 35.7 against 33.0).
+constexpr int kSkWholeTileSlack = 3;
+
 // Clusters of `s` CTAs of `kernel` resident at once on the current device
 // (cached per kernel, cluster size and shared-memory size; 0 if the query
 // fails, which leaves the caller on stream-K).
@@ -394,14 +404,15 @@ q4_status run_gemv(const q4_weight* const* wv, int n, const void* x, int64_t B, 
     const dim3 block((kSkCW + 1 + helpers) * 32);
     auto kernel = two_helpers ? q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 2, false>
                               : q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 1, false>;
-    // the cluster fix-up, when its clusters fit (see kSkClusterSlack)
+    // the cluster fix-up, when its clusters fit (see kSkClusterSlack), else
+    // the whole-tile grid when it fits (see kSkWholeTileSlack), else stream-K
+    const int64_t pmax = static_cast<int64_t>(kSkCtasPerSm) * sm_count(dev);
+    const int64_t sk_iters = (p.T + p.P - 1) / p.P;
     int cluster_s = 1;
     {
         const SkGeom gcl = sk_geom(kSkRT, stages, static_cast<int>(B), SYM, true);
         auto kcl = two_helpers ? q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 2, true>
                                : q4_gemv_sk_kernel<BF16, GS, SYM, kSkCW, 1, true>;
-        const int64_t pmax = static_cast<int64_t>(kSkCtasPerSm) * sm_count(dev);
-        const int64_t sk_iters = (p.T + p.P - 1) / p.P;
         const bool fits = kSkCtasPerSm * (gcl.total + 1024) <= static_cast<size_t>(per_sm);
         for (int S = 8; fits && S >= 2 && cluster_s == 1; --S) {
             if (S > p.nchunks || p.row_tiles * S > pmax) continue;
@@ -414,7 +425,11 @@ q4_status run_gemv(const q4_weight* const* wv, int n, const void* x, int64_t B, 
             }
         }
     }
-    const int64_t grid = cluster_s > 1 ? p.row_tiles * cluster_s : p.P;
+    int64_t grid = p.P;
+    if (cluster_s > 1)
+        grid = p.row_tiles * cluster_s;
+    else if (p.row_tiles <= pmax && p.nchunks <= sk_iters + kSkWholeTileSlack)
+        grid = p.row_tiles;  // T p / P = p nchunks: CTA p owns row tile p whole
     const int64_t G = in / GS;
     // scale / zero windows by TMA when every product's rows are 16-byte aligned
     bool meta_tma = (G % 8) == 0;

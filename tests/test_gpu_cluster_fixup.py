@@ -67,7 +67,7 @@ def test_uneven_split_ragged_tiles(B):
     """1000 rows (7 full tiles and one of 104), in = 3968: 16 chunks, the
     last one half full, over clusters of 8 (two chunks per CTA)."""
     _need_gpu()
-    _case(1000, 3968, 64, False, B, xdtype=torch.float16, ydtype=torch.bfloat16, seed=10 + B)
+    _case(1000, 3968, 64, False, B, xdtype=torch.float16, ydtype=torch.float16, seed=10 + B)
 
 
 @pytest.mark.gpu

@@ -164,13 +164,34 @@ def test_cluster_plans_launched(name, out, inn):
         check_cluster_plan(tiles, nchunks, S)
 
 
+def whole_tile_grid(tiles, nchunks, P, pmax, slack=3):
+    """The library's whole-tile grid (when no cluster plan is taken): one CTA
+    per row tile if the tiles fit the grid and a tile is at most `slack`
+    chunks longer than the longest stream-K range."""
+    return tiles <= pmax and nchunks <= -(-tiles * nchunks // P) + slack
+
+
 def test_cluster_choice_on_the_8b_layer():
     # q/k/v grouped (48 tiles x 16 chunks), o (32 x 16), down (32 x 56):
-    # cluster candidates; gate/up grouped (224 tiles) keeps stream-K
+    # cluster candidates; gate/up grouped (224 tiles) has none and takes the
+    # whole-tile grid (16 chunks against 13); the 70B gate/up (224 x 32
+    # chunks, against 25) stays on stream-K
     assert cluster_size(48, 16, 296, 296) == 6
     assert cluster_size(32, 16, 256, 296) == 8
     assert cluster_size(32, 56, 296, 296) == 8
     assert cluster_size(224, 16, 296, 296) == 1
+    assert whole_tile_grid(224, 16, 296, 296)
+    assert cluster_size(224, 32, 296, 296) == 1 and not whole_tile_grid(224, 32, 296, 296)
+
+
+@pytest.mark.parametrize("tiles,nchunks", [(224, 16), (1, 1), (150, 3), (296, 9)])
+def test_whole_tile_grid_partition(tiles, nchunks):
+    """P = row_tiles: CTA p's range is exactly row tile p, so no segment is
+    partial and the fix-up never runs."""
+    T, P = tiles * nchunks, tiles
+    for p in range(P):
+        assert segments(p, T, P, nchunks) == [(p, 0, nchunks, True)]
+    check_plan(tiles, nchunks, P)
 
 
 def test_random_cluster_plans():
