@@ -290,9 +290,12 @@ SkPlan sk_plan(int64_t out, int64_t in, int sms) {
 // distributed shared memory instead of the workspace, counter and
 // last-arriver pass.  Taken with the largest S <= 8 whose clusters the
 // device holds all at once, unless its CTAs run more than kSkClusterSlack
-// chunks beyond the longest stream-K range; otherwise stream-K.
+// chunks beyond the longest stream-K range; otherwise stream-K.  (Measured:
+// a slack of 2 takes the 70B k_proj, 8 tiles x 32 chunks, from 8.8 to 5.6 us
+// and the 70B q/k/v group from 18.6 to 17.6 us; 3 would also move the 70B
+// down_proj, 28 chunks against 25, which is slower.)
 #ifndef Q4_SK_CLUSTER_SLACK
-#define Q4_SK_CLUSTER_SLACK 1
+#define Q4_SK_CLUSTER_SLACK 2
 #endif
 constexpr int kSkClusterSlack = Q4_SK_CLUSTER_SLACK;
 

@@ -124,7 +124,7 @@ def test_owner_formula_is_the_inverse_of_the_split():
 # being one non-empty partial segment of row tile p // S, the ranks of a tile
 # covering its chunks in rank order.
 
-def cluster_size(tiles, nchunks, P, pmax, slack=1):
+def cluster_size(tiles, nchunks, P, pmax, slack=2):
     """The library's candidate: the largest S <= 8 that fits the grid, unless
     its CTAs run more than `slack` chunks beyond the longest stream-K range.
     (On the device it is then taken only if all row_tiles clusters of S CTAs
@@ -182,6 +182,17 @@ def test_cluster_choice_on_the_8b_layer():
     assert cluster_size(224, 16, 296, 296) == 1
     assert whole_tile_grid(224, 16, 296, 296)
     assert cluster_size(224, 32, 296, 296) == 1 and not whole_tile_grid(224, 32, 296, 296)
+
+
+def test_cluster_choice_on_the_70b_layer():
+    # k_proj / v_proj (8 tiles x 32 chunks, stream-K P = 128): S = 8, 4
+    # chunks per CTA against 2; q/k/v grouped (80 x 32, P = 296): S = 3, 11
+    # against 9; o_proj (64 x 32): S = 4, 8 against 7; down_proj (64 x 112):
+    # 28 against 25 stays on stream-K
+    assert cluster_size(8, 32, 128, 296) == 8
+    assert cluster_size(80, 32, 296, 296) == 3
+    assert cluster_size(64, 32, 296, 296) == 4
+    assert cluster_size(64, 112, 296, 296) == 1
 
 
 @pytest.mark.parametrize("tiles,nchunks", [(224, 16), (1, 1), (150, 3), (296, 9)])
