@@ -13,6 +13,17 @@
 // and resets the counter, so the counters are zero again for the next call.
 // No CTA ever waits for another.
 //
+// The host picks P per shape; the same split then yields two special plans.
+//  * Cluster fix-up (template flag CLUSTER): P = row_tiles x S, launched in
+//    clusters of S <= 8.  CTA p holds K part p % S of row tile p / S, so the
+//    S CTAs of a tile are one cluster.  Each keeps its partial tile in shared
+//    memory, and after a cluster barrier rank r adds rows
+//    [RT r / S, RT (r+1) / S) of the S partials in rank order through
+//    distributed shared memory.  No workspace, counter or atomic.  Every
+//    thread of every CTA passes both cluster barriers.
+//  * Whole-tile grid: P = row_tiles, every range one whole tile, y stored
+//    directly (the stream-K instance; its fix-up path is never reached).
+//
 // Launch overlap: the kernel lets the next kernel of the stream launch as
 // soon as it has started (programmatic dependent launch), and itself issues
 // the loads of its first stages of weights and scales -- which no preceding
