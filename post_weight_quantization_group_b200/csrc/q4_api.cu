@@ -819,6 +819,24 @@ SkPlan fp4_plan(int64_t out, int64_t in, int64_t B, int sms) {
     return stream_k_plan(out, in, kF4RT, sms, kF4MinIters, f4_nt(B), kF4ChunkCodes);
 }
 
+// Cluster plan of the tcgen05 products (FP4, bf16 reference) for activation
+// tiles NT >= 64, whose stream-K final epilogue (an NT x 128 fp32 partial per
+// CTA stored, counted and summed by the last arriver) costs the most: the
+// largest S <= 8 with row_tiles x S CTAs all resident, each CTA at most 25 %
+// longer than the longest stream-K range.  Returns 1 for stream-K.
+template <typename Kern>
+int tc_cluster_size(Kern kcl, const SkPlan& p, int nt, size_t smem, int64_t pmax) {
+    if (nt < 64) return 1;
+    const int64_t sk_iters = (p.T + p.P - 1) / p.P;
+    for (int S = 8; S >= 2; --S) {
+        if (S > p.nchunks || p.row_tiles * S > pmax) continue;
+        if ((p.nchunks + S - 1) / S * 4 > sk_iters * 5) return 1;
+        if (!set_kernel_attrs(kcl, static_cast<int>(smem), false)) return 1;
+        if (max_active_clusters(kcl, S, dim3(kF4Threads), smem) >= p.row_tiles) return S;
+    }
+    return 1;
+}
+
 template <bool NV, int NT>
 q4_status run_fp4(const uint8_t* wq, const uint8_t* wsc, const float* wts, int64_t out,
                   int64_t in, const uint8_t* xq, const uint8_t* xsc, const float* xts, int64_t B,
@@ -846,16 +864,20 @@ q4_status run_fp4(const uint8_t* wq, const uint8_t* wsc, const float* wts, int64
         !make_tmap_2d(&tmap_sx, xsc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(B),
                       sb, NT, SFB, CU_TENSOR_MAP_SWIZZLE_NONE))
         return Q4_ERR_CUDA;
-    auto kernel = fp4_gemm_tc_kernel<NV, NT>;
+    const int cluster_s = tc_cluster_size(fp4_gemm_tc_kernel<NV, NT, true>, p, NT, geo.total,
+                                          sm_count(dev));
+    auto kernel = cluster_s > 1 ? fp4_gemm_tc_kernel<NV, NT, true> : fp4_gemm_tc_kernel<NV, NT, false>;
+    const int64_t grid = cluster_s > 1 ? p.row_tiles * cluster_s : p.P;
     if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), false)) return Q4_ERR_CUDA;
     unsigned* status = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
         return Q4_ERR_CUDA;
     unsigned* ws_count = reinterpret_cast<unsigned*>(ws);
     float* ws_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kWsCounterBytes);
-    return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3(kF4Threads), geo.total, 1,
-                     true, st, tmap_w, tmap_sw, tmap_x, tmap_sx, wts, xts, stages,
-                     static_cast<int>(B), out, p.nchunks, p.T, y, ydt, ws_part, ws_count, status);
+    return launch_ex(kernel, dim3(static_cast<unsigned>(grid)), dim3(kF4Threads), geo.total,
+                     cluster_s, true, st, tmap_w, tmap_sw, tmap_x, tmap_sx, wts, xts, stages,
+                     static_cast<int>(B), out, p.nchunks, p.T, y, ydt, ws_part, ws_count, status,
+                     cluster_s);
 }
 
 SkPlan bf16_plan(int64_t out, int64_t in, int64_t B, int sms) {
@@ -882,16 +904,19 @@ q4_status run_bf16_tc(const void* W, int64_t out, int64_t in, const void* x, int
         !make_tmap_2d(&tmap_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, static_cast<uint64_t>(B),
                       static_cast<uint64_t>(in), NT, kBoxElems))
         return Q4_ERR_CUDA;
-    auto kernel = bf16_gemm_tc_kernel<NT>;
+    const int cluster_s = tc_cluster_size(bf16_gemm_tc_kernel<NT, true>, p, NT, geo.total,
+                                          sm_count(dev));
+    auto kernel = cluster_s > 1 ? bf16_gemm_tc_kernel<NT, true> : bf16_gemm_tc_kernel<NT, false>;
+    const int64_t grid = cluster_s > 1 ? p.row_tiles * cluster_s : p.P;
     if (!set_kernel_attrs(kernel, static_cast<int>(geo.total), false)) return Q4_ERR_CUDA;
     unsigned* status = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_q4_status) != cudaSuccess)
         return Q4_ERR_CUDA;
     unsigned* ws_count = reinterpret_cast<unsigned*>(ws);
     float* ws_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kWsCounterBytes);
-    return launch_ex(kernel, dim3(static_cast<unsigned>(p.P)), dim3(kF4Threads), geo.total, 1,
-                     true, st, tmap_w, tmap_x, stages, static_cast<int>(B), out, p.nchunks, p.T,
-                     y, 1, ws_part, ws_count, status);
+    return launch_ex(kernel, dim3(static_cast<unsigned>(grid)), dim3(kF4Threads), geo.total,
+                     cluster_s, true, st, tmap_w, tmap_x, stages, static_cast<int>(B), out,
+                     p.nchunks, p.T, y, 1, ws_part, ws_count, status, cluster_s);
 }
 
 template <bool NV>

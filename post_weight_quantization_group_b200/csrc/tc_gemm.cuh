@@ -240,7 +240,11 @@ __device__ __forceinline__ void gather_scales(uint32_t tile, int lane, int nrows
     }
 }
 
-template <int KIND, int NT>
+// CLUSTER: the grid is row_tiles x cluster_s CTAs in clusters of cluster_s,
+// CTA p holding K part p % cluster_s of row tile p / cluster_s (one partial
+// segment each); the cluster adds its partials through distributed shared
+// memory instead of the workspace protocol.
+template <int KIND, int NT, bool CLUSTER>
 __device__ __forceinline__ void tc_gemm_body(const CUtensorMap& tmap_w, const CUtensorMap& tmap_sw,
                                              const CUtensorMap& tmap_x, const CUtensorMap& tmap_sx,
                                              const float* __restrict__ w_ts,
@@ -249,7 +253,7 @@ __device__ __forceinline__ void tc_gemm_body(const CUtensorMap& tmap_w, const CU
                                              void* __restrict__ y, int ydt,
                                              float* __restrict__ ws_part,
                                              unsigned* __restrict__ ws_count,
-                                             unsigned* __restrict__ status) {
+                                             unsigned* __restrict__ status, int cluster_s) {
     using K = TcKind<KIND>;
     constexpr bool NV = K::NV;
     constexpr int SFB = K::sf_bytes;
@@ -479,6 +483,27 @@ __device__ __forceinline__ void tc_gemm_body(const CUtensorMap& tmap_w, const CU
                                        kWaitLimitNs);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
+            if constexpr (CLUSTER) {
+                // The CTA's one (partial) segment: its accumulator goes to the
+                // drained pipeline's shared memory, [NT columns x 128 rows]
+                // fp32, for the cluster's reduction after the role branches.
+                if (ok) {
+#pragma unroll 1
+                    for (int c0 = 0; c0 < NT; c0 += PW) {
+                        uint32_t v[PW];
+                        tmem_ld_cols<PW>(tl + static_cast<uint32_t>(a * NT + c0), v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < PW; ++e)
+                            sts32(fix_smem + static_cast<uint32_t>(((c0 + e) * kF4RT + r) * 4), v[e]);
+                    }
+                }
+                c += len;
+                chunk = 0;
+                ++tile;
+                ++seg;
+                continue;
+            }
             const int64_t row = static_cast<int64_t>(tile) * kF4RT + r;
             const int slot = static_cast<int>(2 * p + (first ? 0 : 1));
             float* part = ws_part + static_cast<size_t>(slot) * kF4RT * NT;
@@ -637,6 +662,45 @@ __device__ __forceinline__ void tc_gemm_body(const CUtensorMap& tmap_w, const CU
 
     tc_fence_before();
     __syncthreads();
+    if constexpr (CLUSTER) {
+        // Every thread of every CTA of the cluster passes both barriers: all
+        // roles have joined at the __syncthreads above.
+        cluster_sync_all();  // every rank's partial is in its shared memory
+        if (warp >= 6) {
+            // rank rk writes y for columns [NT rk / S, NT (rk+1) / S) of the
+            // tile, adding the S partials in rank order
+            const int S = cluster_s;
+            const int rk = static_cast<int>(cluster_ctarank());
+            const int r = 32 * (warp & 3) + lane;
+            const int64_t row = static_cast<int64_t>(tile0) * kF4RT + r;
+            const float g = NV ? __ldg(w_ts) * __ldg(x_ts) : 1.0f;
+            const uint32_t base = smem_u32(smem);
+            const int n_end = min(NT * (rk + 1) / S, B);
+            constexpr int U = 8;
+            for (int n0 = NT * rk / S; n0 < n_end; n0 += U) {
+                float acc[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) acc[u] = 0.f;
+                for (int k = 0; k < S; ++k) {
+                    float v[U];
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int n = min(n0 + u, NT - 1);
+                        v[u] = ld_shared_cluster_f32(mapa_shared(
+                            base + static_cast<uint32_t>((n * kF4RT + r) * 4), static_cast<uint32_t>(k)));
+                    }
+#pragma unroll
+                    for (int u = 0; u < U; ++u) acc[u] += v[u];
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (n0 + u < n_end && row < out)
+                        store_y(y, ydt, static_cast<int64_t>(n0 + u) * out + row, g * acc[u]);
+            }
+        }
+        __syncwarp();
+        cluster_sync_all();  // no rank leaves while another still reads it
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tbase, kF4TmemCols);
@@ -644,7 +708,7 @@ __device__ __forceinline__ void tc_gemm_body(const CUtensorMap& tmap_w, const CU
 }
 
 // W4A4 product of two FP4 operands (NVFP4 or MXFP4).
-template <bool NV, int NT>
+template <bool NV, int NT, bool CLUSTER>
 __global__ void __launch_bounds__(kF4Threads, 1)
     fp4_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ CUtensorMap tmap_sw,
@@ -653,22 +717,24 @@ __global__ void __launch_bounds__(kF4Threads, 1)
                        const float* __restrict__ w_ts, const float* __restrict__ x_ts, int stages,
                        int B, int64_t out, int nchunks, int64_t T, void* __restrict__ y, int ydt,
                        float* __restrict__ ws_part, unsigned* __restrict__ ws_count,
-                       unsigned* __restrict__ status) {
-    tc_gemm_body<NV ? kKindNVFP4 : kKindMXFP4, NT>(tmap_w, tmap_sw, tmap_x, tmap_sx, w_ts, x_ts,
-                                                   stages, B, out, nchunks, T, y, ydt, ws_part,
-                                                   ws_count, status);
+                       unsigned* __restrict__ status, int cluster_s) {
+    tc_gemm_body<NV ? kKindNVFP4 : kKindMXFP4, NT, CLUSTER>(tmap_w, tmap_sw, tmap_x, tmap_sx, w_ts,
+                                                            x_ts, stages, B, out, nchunks, T, y,
+                                                            ydt, ws_part, ws_count, status,
+                                                            cluster_s);
 }
 
 // The bf16 reference product y = x W^T (bf16 W and x, fp32 accumulation).
-template <int NT>
+template <int NT, bool CLUSTER>
 __global__ void __launch_bounds__(kF4Threads, 1)
     bf16_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
                         const __grid_constant__ CUtensorMap tmap_x, int stages, int B, int64_t out,
                         int nchunks, int64_t T, void* __restrict__ y, int ydt,
                         float* __restrict__ ws_part, unsigned* __restrict__ ws_count,
-                        unsigned* __restrict__ status) {
-    tc_gemm_body<kKindBF16, NT>(tmap_w, tmap_w, tmap_x, tmap_x, nullptr, nullptr, stages, B, out,
-                                nchunks, T, y, ydt, ws_part, ws_count, status);
+                        unsigned* __restrict__ status, int cluster_s) {
+    tc_gemm_body<kKindBF16, NT, CLUSTER>(tmap_w, tmap_w, tmap_x, tmap_x, nullptr, nullptr, stages,
+                                         B, out, nchunks, T, y, ydt, ws_part, ws_count, status,
+                                         cluster_s);
 }
 
 }  // namespace q4dev
