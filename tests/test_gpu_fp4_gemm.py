@@ -145,6 +145,34 @@ def test_fp4_gemm_deterministic_split_tiles(fmt):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("fmt,inn,B", [("nvfp4", 4096, 64), ("mxfp4", 2560, 100),
+                                       ("nvfp4", 1536, 33)])
+def test_fp4_gemm_cluster_fixup(fmt, inn, B):
+    """B > 32 on 300 rows: the CTAs of a row tile form a cluster (8 chunks of
+    K -> 8 CTAs of one chunk each, 5 -> 5, 3 -> 3) and add their partials
+    through distributed shared memory; every row checked, repeated calls
+    bit-identical."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    W, X, y = _product_case(fmt, 300, inn, B, seed=600 + B, nrows=300)
+    for _ in range(2):
+        assert torch.equal(q4.fp4_gemm(W, X, y_dtype=torch.float32), y)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_fp4_gemm_cluster_deterministic_70b(fmt):
+    """70B down_proj at B = 128: 64 row tiles x 2 CTAs in clusters of two;
+    repeated calls agree bit for bit."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    out, inn = wl.LLAMA3_70B["down_proj"]
+    W, X, y = _product_case(fmt, out, inn, 128, seed=700, nrows=16)
+    for _ in range(2):
+        assert torch.equal(q4.fp4_gemm(W, X, y_dtype=torch.float32), y)
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
 def test_fp4_gemm_end_to_end_quantized(fmt):
     """Weights N(0, 0.02^2) and activations with outlier channels, each
