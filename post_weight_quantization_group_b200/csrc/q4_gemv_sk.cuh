@@ -591,9 +591,17 @@ __global__ void __launch_bounds__((CW + 1 + NH) * 32, 2)
         const int v_end = (RT * (r + 1) / S) * 8;
         for (int v = (RT * r / S) * 8 + static_cast<int>(threadIdx.x); v < v_end; v += CW * 32) {
             const int row = v >> 3, col = v & 7;
+            // all S remote loads in flight at once, then the sum in rank order
+            float part[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                part[q] = q < S ? ld_shared_cluster_f32(mapa_shared(red + static_cast<uint32_t>(v) * 4,
+                                                                    static_cast<uint32_t>(q)))
+                                : 0.f;
             float sum = 0.f;
-            for (int q = 0; q < S; ++q)
-                sum += ld_shared_cluster_f32(mapa_shared(red + static_cast<uint32_t>(v) * 4, q));
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (q < S) sum += part[q];
             if (col < B && row0 + row < out)
                 store_y(y, ydt, static_cast<int64_t>(col) * out + row0 + row, sum);
         }
