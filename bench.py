@@ -51,12 +51,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of q4_gemv_sk_kernel per algorithmic byte, from the ncu
 # capture of the four launches of one Llama-3-8B layer as the step launches
 # them (q/k/v grouped, o, gate/up grouped, down): dram__bytes_read.sum +
-# dram__bytes_write.sum = 112.88 MB against 112.62 MB of algorithmic bytes
+# dram__bytes_write.sum = 112.70 MB against 112.62 MB of algorithmic bytes
 # (q/k/v, o and down with the cluster fix-up, gate/up on the whole-tile
 # grid).  Scaled to the step's average launch; it must be re-taken whenever
 # the kernel or its launch plan changes.
-GEMV_TRAFFIC_RATIO = 112.876544 / 112.623616
-GEMV_TRAFFIC_SOURCE = ("ncu --set full on the 4 launches of one B=1 layer "
+GEMV_TRAFFIC_RATIO = 112.698368 / 112.623616
+GEMV_TRAFFIC_SOURCE = ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum on the 4 "
+                       "launches of one B=1 layer "
                        "(profiles/q4_gemv_sk_llama3_8b_layer_grouped_full.txt)")
 
 
