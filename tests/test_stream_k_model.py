@@ -212,3 +212,38 @@ def test_random_cluster_plans():
         nchunks = rng.randint(S, 80)
         tiles = rng.randint(1, 296 // S)
         check_cluster_plan(tiles, nchunks, S)
+
+
+# ------------------------------------------- tcgen05 products (FP4, bf16)
+def tc_cluster_size(tiles, nchunks, nt, pmax=148, min_iters=4):
+    """The FP4 / bf16 products' candidate: only for activation tiles nt >= 64,
+    the largest S <= 8 with tiles x S CTAs (one per SM), each CTA's range at
+    most 25 % longer than the longest stream-K range.  (On the device it is
+    then taken only if all clusters are resident at once.)"""
+    if nt < 64:
+        return 1
+    T = tiles * nchunks
+    P = stream_k_P(T, pmax, min_iters)
+    sk = -(-T // P)
+    for S in range(8, 1, -1):
+        if S > nchunks or tiles * S > pmax:
+            continue
+        return S if -(-nchunks // S) * 4 <= sk * 5 else 1
+    return 1
+
+
+def test_tc_cluster_choice_on_70b_shapes():
+    # FP4 chunks are 512 codes, bf16 chunks 128 values; 128-row tiles
+    assert tc_cluster_size(64, 56, 128) == 2    # FP4 down_proj, B > 64: 28 against 25
+    assert tc_cluster_size(64, 56, 64) == 2     # FP4 down_proj, 33 <= B <= 64
+    assert tc_cluster_size(64, 56, 32) == 1     # NT <= 32: stream-K
+    assert tc_cluster_size(224, 16, 128) == 1   # FP4 gate_proj: 224 tiles > 148 SMs
+    assert tc_cluster_size(64, 224, 128) == 2   # bf16 down_proj: 112 against 97
+    assert tc_cluster_size(64, 16, 128) == 2    # FP4 q_proj: 8 against 7
+
+
+@pytest.mark.parametrize("tiles,nchunks", [(3, 8), (3, 5), (3, 3), (64, 56), (64, 224)])
+def test_tc_cluster_partition(tiles, nchunks):
+    S = tc_cluster_size(tiles, nchunks, 128)
+    assert S > 1
+    check_cluster_plan(tiles, nchunks, S)
