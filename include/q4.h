@@ -327,7 +327,9 @@ Q4_API q4_status q4_gemv_noalloc(const q4_weight* w, const void* x, q4_dtype x_d
  *              aligned, zero-filled before its first use (the kernel leaves
  *              its counters zero again); the same layout as the INT4
  *              products' workspace, so one buffer serves both.
- * Deterministic: split tiles add their partials in a fixed order.
+ * Deterministic: split tiles add their partials in a fixed order (through the
+ * workspace, or, for B > 32 when the row tiles x S CTAs fit the device,
+ * through distributed shared memory inside clusters of S CTAs).
  */
 Q4_API size_t bf16_ref_workspace_bytes(int64_t out, int64_t in, int64_t B);
 Q4_API q4_status bf16_gemv_ref_bw(const void* W, int64_t out, int64_t in, const void* x, int64_t B,
@@ -451,7 +453,9 @@ Q4_API q4_status nvfp4_dequant(const uint8_t* packed, const uint8_t* scales,
  *                   first use (the kernels leave it zeroed again); one call
  *                   at a time per workspace
  * Accumulation is fp32 inside the tensor core; the result is deterministic
- * (split tiles add their partials in a fixed order).  B > 128 runs as slices
+ * (split tiles add their partials in a fixed order: through the workspace,
+ * or, for B > 32 when the row tiles x S CTAs fit the device, through
+ * distributed shared memory inside clusters of S CTAs).  B > 128 runs as slices
  * of 128 activation rows.  Errors: Q4_ERR_INVALID_ARG (format, dtype, null
  * pointer), Q4_ERR_SHAPE, Q4_ERR_ALIGNMENT, Q4_ERR_WORKSPACE; a device-side
  * wait that runs out sets Q4_ERR_TIMEOUT for q4_sync_status.
